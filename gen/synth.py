@@ -1,0 +1,170 @@
+"""Seeded synthetic inputs for the GPT-OSS MXFP4 MoE feed-forward layer.
+
+This module draws random numbers and lays them out in the layer's storage
+format. It holds none of the layer's arithmetic: no dequantisation, no router,
+no activation. The one place where inputs depend on the layer (rejecting tokens
+whose top-k router logits are too close to call) is delegated to a caller-given
+``margin_fn``, so the generator itself stays method-free. Both the float64
+oracle tests and the GPU harness read their inputs from here.
+
+Storage format (all arrays C-contiguous, row-major):
+
+  x               uint16 [T, H]           bf16 bit patterns
+  router_w        float32 [E, H]
+  router_b        float32 [E]
+  gate_up_blocks  uint8  [E, 2I, H/32, 16] two E2M1 codes per byte, low nibble first
+  gate_up_scales  uint8  [E, 2I, H/32]     E8M0 exponents, one per 32-element block
+  gate_up_bias    uint16 [E, 2I]           bf16 bits, gate/up rows interleaved
+  down_blocks     uint8  [E, H, I/32, 16]
+  down_scales     uint8  [E, H, I/32]
+  down_bias       uint16 [E, H]            bf16 bits
+
+The gate_up orientation [E, 2I, H] (output rows, reduction columns) is the one
+MXFP4-dequantised checkpoints use per the Megatron-Bridge GPT-OSS bridge docs
+(``maybe_modify_loaded_hf_weight``); down is [E, H, I] likewise.
+
+Distribution reading: ``N(0, 1/H)`` for the router weight is a variance of 1/H
+(standard deviation H**-0.5, the fan-in convention, which makes router logits
+O(1)); ``N(0, 0.1)`` and ``N(0, 0.02)`` for the biases give the standard
+deviation, as numpy's ``normal(loc, scale)`` does.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Callable, Dict, Optional
+
+import numpy as np
+
+__all__ = ["Config", "CONFIGS", "make_inputs", "f32_to_bf16_bits", "INPUT_ORDER"]
+
+
+@dataclasses.dataclass(frozen=True)
+class Config:
+    name: str
+    T: int
+    H: int
+    I: int
+    E: int
+    k: int
+    scale_lo: int
+    scale_hi: int
+    router_bias: str  # "normal" (N(0, 0.1)) or "zipf" (log of Zipf(1.2) popularity)
+    zipf_s: float = 1.2
+
+    @property
+    def packed_bytes_per_expert(self) -> int:
+        """Packed MXFP4 bytes (blocks + scales) of one expert's gate_up and down."""
+        gu = 2 * self.I * (self.H // 2 + self.H // 32)
+        dn = self.H * (self.I // 2 + self.I // 32)
+        return gu + dn
+
+    @property
+    def bias_bytes_per_expert(self) -> int:
+        return 2 * (2 * self.I + self.H)
+
+
+# The five synthetic workloads: a tiny layer and gpt-oss-20b / -120b shaped layers
+# (sizes from the ZeroModels GPT-OSS docs: embed_dim 2880, mlp_dim 2880, 32 / 128
+# experts, num_experts_per_tok 4).
+CONFIGS: Dict[str, Config] = {
+    c.name: c
+    for c in (
+        Config("tiny", T=16, H=256, I=256, E=8, k=2, scale_lo=119, scale_hi=123, router_bias="normal"),
+        Config("gpt-oss-20b-decode", T=8, H=2880, I=2880, E=32, k=4, scale_lo=118, scale_hi=122,
+               router_bias="normal"),
+        Config("gpt-oss-20b-prefill", T=4096, H=2880, I=2880, E=32, k=4, scale_lo=118, scale_hi=122,
+               router_bias="normal"),
+        Config("gpt-oss-120b-decode", T=64, H=2880, I=2880, E=128, k=4, scale_lo=118, scale_hi=122,
+               router_bias="normal"),
+        Config("gpt-oss-120b-prefill-zipf", T=8192, H=2880, I=2880, E=128, k=4, scale_lo=118,
+               scale_hi=122, router_bias="zipf"),
+    )
+}
+
+# Order in which arrays are drawn from the generator (and the C-ABI argument order).
+INPUT_ORDER = (
+    "x", "router_w", "router_b",
+    "gate_up_blocks", "gate_up_scales", "gate_up_bias",
+    "down_blocks", "down_scales", "down_bias",
+)
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to bf16 (round to nearest, ties to even); return the bit patterns."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    bias = ((u >> 16) & 1) + 0x7FFF
+    return ((u + bias) >> 16).astype(np.uint16)
+
+
+def _bytes(rng: np.random.Generator, shape) -> np.ndarray:
+    return rng.integers(0, 256, size=shape, dtype=np.uint8)
+
+
+def _scales(rng: np.random.Generator, shape, lo: int, hi: int) -> np.ndarray:
+    return rng.integers(lo, hi + 1, size=shape, dtype=np.uint8)
+
+
+def zipf_router_bias(E: int, s: float) -> np.ndarray:
+    """router_b[e] = log p_e with p_e proportional to (e+1)^-s (expert e has popularity rank e+1)."""
+    p = (np.arange(1, E + 1, dtype=np.float64)) ** (-s)
+    p /= p.sum()
+    return np.log(p).astype(np.float32)
+
+
+MarginFn = Callable[[np.ndarray, np.ndarray, np.ndarray, int], np.ndarray]
+
+
+def make_inputs(
+    cfg: "Config | str",
+    seed: int = 0,
+    margin_fn: Optional[MarginFn] = None,
+    min_margin: float = 1e-3,
+    max_attempts: int = 1000,
+    T: Optional[int] = None,
+) -> Dict[str, np.ndarray]:
+    """Draw one layer's inputs.
+
+    ``margin_fn(x_bits, router_w, router_b, k)`` must return, per token, the smallest
+    gap between adjacent logits among the k+1 largest (float64). Tokens whose gap is
+    below ``min_margin`` get their x row redrawn from the sub-stream
+    ``default_rng([seed, 1, t, attempt])`` until every token passes, so that the
+    top-k set and its order are unambiguous. Without ``margin_fn`` no token is redrawn.
+    ``T`` overrides the config's token count (the x draw then changes accordingly).
+    """
+    if isinstance(cfg, str):
+        cfg = CONFIGS[cfg]
+    T = cfg.T if T is None else int(T)
+    H, I, E, k = cfg.H, cfg.I, cfg.E, cfg.k
+    if H % 32 or I % 32:
+        raise ValueError("H and I must be multiples of the 32-element MX block")
+    rng = np.random.default_rng(seed)
+    out: Dict[str, np.ndarray] = {}
+    out["x"] = f32_to_bf16_bits(rng.standard_normal((T, H), dtype=np.float32))
+    out["router_w"] = (rng.standard_normal((E, H), dtype=np.float32) * np.float32(1.0 / np.sqrt(H))).astype(
+        np.float32)
+    if cfg.router_bias == "zipf":
+        out["router_b"] = zipf_router_bias(E, cfg.zipf_s)
+    else:
+        out["router_b"] = (rng.standard_normal(E, dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+    out["gate_up_blocks"] = _bytes(rng, (E, 2 * I, H // 32, 16))
+    out["gate_up_scales"] = _scales(rng, (E, 2 * I, H // 32), cfg.scale_lo, cfg.scale_hi)
+    out["gate_up_bias"] = f32_to_bf16_bits(rng.standard_normal((E, 2 * I), dtype=np.float32) * np.float32(0.02))
+    out["down_blocks"] = _bytes(rng, (E, H, I // 32, 16))
+    out["down_scales"] = _scales(rng, (E, H, I // 32), cfg.scale_lo, cfg.scale_hi)
+    out["down_bias"] = f32_to_bf16_bits(rng.standard_normal((E, H), dtype=np.float32) * np.float32(0.02))
+
+    if margin_fn is not None:
+        x = out["x"]
+        bad = np.nonzero(margin_fn(x, out["router_w"], out["router_b"], k) < min_margin)[0]
+        attempt = 0
+        while bad.size:
+            if attempt >= max_attempts:
+                raise RuntimeError(f"{bad.size} tokens still below the router margin after {attempt} redraws")
+            for t in bad:
+                sub = np.random.default_rng([seed, 1, int(t), attempt])
+                x[t] = f32_to_bf16_bits(sub.standard_normal(H, dtype=np.float32))
+            m = margin_fn(x[bad], out["router_w"], out["router_b"], k)
+            bad = bad[m < min_margin]
+            attempt += 1
+    return out

@@ -1,0 +1,63 @@
+"""The seeded input generator: shapes, determinism, distributions and the router-margin redraw."""
+
+import ml_dtypes
+import numpy as np
+import pytest
+
+import oracle
+from gen.synth import CONFIGS, Config, f32_to_bf16_bits, make_inputs, zipf_router_bias
+
+
+def test_shapes_dtypes_tiny():
+    c = CONFIGS["tiny"]
+    d = make_inputs("tiny")
+    assert d["x"].shape == (c.T, c.H) and d["x"].dtype == np.uint16
+    assert d["router_w"].shape == (c.E, c.H) and d["router_w"].dtype == np.float32
+    assert d["router_b"].shape == (c.E,)
+    assert d["gate_up_blocks"].shape == (c.E, 2 * c.I, c.H // 32, 16) and d["gate_up_blocks"].dtype == np.uint8
+    assert d["gate_up_scales"].shape == (c.E, 2 * c.I, c.H // 32)
+    assert d["gate_up_bias"].shape == (c.E, 2 * c.I) and d["gate_up_bias"].dtype == np.uint16
+    assert d["down_blocks"].shape == (c.E, c.H, c.I // 32, 16)
+    assert d["down_scales"].shape == (c.E, c.H, c.I // 32)
+    assert d["down_bias"].shape == (c.E, c.H)
+    assert d["gate_up_scales"].min() >= c.scale_lo and d["gate_up_scales"].max() <= c.scale_hi
+
+
+def test_deterministic_and_seed_sensitive():
+    a = make_inputs("tiny", seed=0)
+    b = make_inputs("tiny", seed=0)
+    c = make_inputs("tiny", seed=1)
+    for k in a:
+        assert np.array_equal(a[k], b[k])
+    assert not np.array_equal(a["x"], c["x"])
+
+
+def test_bf16_rounding_is_rne():
+    f = np.array([1.0, 1.00390625, 1.005859375, 1.0078125 + 2 ** -9, -3.14159], np.float32)
+    assert np.array_equal(f32_to_bf16_bits(f), f.astype(ml_dtypes.bfloat16).view(np.uint16))
+
+
+def test_margin_redraw_makes_every_token_pass():
+    inp = make_inputs("tiny", margin_fn=oracle.router_margins, min_margin=0.05)
+    m = oracle.router_margins(inp["x"], inp["router_w"], inp["router_b"], CONFIGS["tiny"].k)
+    assert m.min() >= 0.05
+    raw = make_inputs("tiny")
+    assert not np.array_equal(raw["x"], inp["x"])  # some tokens were redrawn at this margin
+
+
+def test_zipf_bias_skews_routing():
+    b = zipf_router_bias(128, 1.2)
+    p = np.exp(b.astype(np.float64))
+    assert abs(p.sum() - 1) < 1e-6 and np.all(np.diff(b) < 0)
+
+
+def test_distributions_roughly_as_stated():
+    cfg = Config("dist", T=256, H=512, I=64, E=16, k=2, scale_lo=118, scale_hi=122, router_bias="normal")
+    d = make_inputs(cfg, seed=3)
+    x = d["x"].view(ml_dtypes.bfloat16).astype(np.float64)
+    assert abs(x.std() - 1) < 0.02
+    assert abs(d["router_w"].std() * np.sqrt(cfg.H) - 1) < 0.05
+    gb = d["gate_up_bias"].view(ml_dtypes.bfloat16).astype(np.float64)
+    assert abs(gb.std() - 0.02) < 0.003
+    counts = np.bincount(d["gate_up_blocks"].ravel(), minlength=256)
+    assert counts.min() > 0.8 * counts.mean()
