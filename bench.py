@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the GPT-OSS MXFP4 MoE feed-forward layer on B200.
+
+One step = one full layer call (router, top-k, softmax, permutation, gate_up +
+SwiGLU, down, weighted combine) on one batch of synthetic tokens resident in
+HBM. Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Default workload: the gpt-oss-20b-shaped decode layer (T=8, H=I=2880, E=32,
+top-4). L2 is flushed (a 256 MiB write) before every timed step; each step is
+timed with its own CUDA events on the launching stream and the per-step times
+are summed. Under torchrun every rank runs an independent replica on its own
+GPU (no collective on the data path: weak scaling); the reported time is the
+max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gen.synth import CONFIGS, make_inputs  # noqa: E402
+
+DEFAULT_CONFIG = "gpt-oss-20b-decode"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return PEAKS_FALLBACK, "fallback"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--path", type=int, default=0, help="0 auto, 1 decode GEMV, 2 grouped GEMM")
+    ap.add_argument("--decode-kernel", type=int, default=1, help="decode GEMV engine: 0 CUDA-core FMA, 1 warp MMA")
+    ap.add_argument("--no-extra", action="store_true", help="skip the prefill side measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- algorithmic units
+
+def layer_units(cfg, n_touched: int, T: int):
+    """Algorithmic bytes and FLOPs of one layer call (dequant work, intermediates and padding excluded)."""
+    H, I, E, k = cfg.H, cfg.I, cfg.E, cfg.k
+    per_expert = cfg.packed_bytes_per_expert + cfg.bias_bytes_per_expert
+    bytes_alg = n_touched * per_expert + E * H * 4 + E * 4 + 2 * T * H * 2
+    flops_alg = 2 * T * k * (2 * I * H + I * H) + 2 * T * E * H
+    return bytes_alg, flops_alg
+
+
+def gateup_units(cfg, n_touched: int, T: int):
+    """Algorithmic bytes / FLOPs of the gate_up stage: touched experts' packed gate_up weights + bias,
+    the token rows in, the SwiGLU rows out."""
+    H, I, k = cfg.H, cfg.I, cfg.k
+    w = n_touched * (2 * I * (H // 2 + H // 32) + 2 * I * 2)
+    bytes_alg = w + T * H * 2 + T * k * I * 2
+    flops = 2 * T * k * 2 * I * H
+    return bytes_alg, flops
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every ~2 ms in a background thread."""
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_sm = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, keep going
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        nv = self.nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "applications_clocks_setting": getattr(nv, "nvmlClocksEventReasonApplicationsClocksSetting", 0x2),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sync_boost": getattr(nv, "nvmlClocksEventReasonSyncBoost", 0x10),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        reasons = set()
+        for _, rs in self.samples:
+            for n, bit in names.items():
+                if rs & bit and n != "gpu_idle":
+                    reasons.add(n)
+        sm = [s for s, _ in self.samples]
+        return {"sm_mhz": float(statistics.median(sm)) if sm else None, "sm_max_mhz": float(self.max_sm),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def upload(inputs, torch):
+    d = {}
+    for k, v in inputs.items():
+        a = np.ascontiguousarray(v)
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        d[k] = torch.from_numpy(a).cuda()
+    return d
+
+
+def weights_list(dev):
+    return [dev[n] for n in ("router_w", "router_b", "gate_up_blocks", "gate_up_scales", "gate_up_bias",
+                             "down_blocks", "down_scales", "down_bias")]
+
+
+def measure(moe, torch, cfg, dev, T, steps, warmup, path, flush, sampler=None, decode_kernel=1):
+    """Time `steps` layer calls; returns dict with per-step ms list, stage ms (summed), n_touched."""
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
+    try:
+        moe.moe_set_option(h, moe.MOE_OPT_PATH, path)
+        moe.moe_set_option(h, moe.MOE_OPT_DECODE_KERNEL, decode_kernel)
+        out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device="cuda")
+        W = weights_list(dev)
+        st = torch.cuda.current_stream()
+        for _ in range(warmup):
+            flush.zero_()
+            moe.moe_forward(h, dev["x"], *W, T, out)
+        # routing of this batch: number of experts touched (for the algorithmic byte count)
+        idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+        moe.moe_debug_route(h, dev["x"], dev["router_w"], dev["router_b"], T, idx)
+        torch.cuda.synchronize()
+        n_touched = int(torch.unique(idx).numel())
+        moe.moe_set_option(h, moe.MOE_OPT_STAGE_EVENTS, steps)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        torch.cuda.synchronize()
+        ctx = sampler if sampler is not None else _Null()
+        with ctx:
+            for i in range(steps):
+                flush.zero_()
+                evs[i][0].record(st)
+                moe.moe_forward(h, dev["x"], *W, T, out)
+                evs[i][1].record(st)
+            torch.cuda.synchronize()
+        step_ms = [a.elapsed_time(b) for a, b in evs]
+        stage_ms, ncalls = moe.moe_stage_times(h)
+        status = moe.moe_sync_status(h)
+        if status != moe.MOE_OK:
+            raise RuntimeError(f"device status {moe.moe_status_string(status)}")
+    finally:
+        moe.moe_destroy(h)
+    return {"step_ms": step_ms, "stage_ms": [s / max(ncalls, 1) for s in stage_ms], "n_touched": n_touched,
+            "out": out}
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def measure_e2e(moe, torch, cfg, dev, x_np, T, steps, warmup, path, flush, decode_kernel=1):
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
+    try:
+        moe.moe_set_option(h, moe.MOE_OPT_PATH, path)
+        moe.moe_set_option(h, moe.MOE_OPT_DECODE_KERNEL, decode_kernel)
+        W = weights_list(dev)
+        x_host = torch.from_numpy(np.ascontiguousarray(x_np).view(np.int16)).pin_memory()
+        out_host = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
+        st = torch.cuda.current_stream()
+        for _ in range(warmup):
+            moe.moe_forward_hostio(h, x_host, *W, T, out_host)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(st)
+            moe.moe_forward_hostio(h, x_host, *W, T, out_host)  # copies in, computes, copies out, syncs
+            evs[i][1].record(st)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_destroy(h)
+    ms = [a.elapsed_time(b) for a, b in evs]
+    return ms, T * cfg.H * 2, T * cfg.H * 2
+
+
+def cpu_baseline(cfg, inputs, budget_s=10.0):
+    """The float64 oracle as it stands, on a bounded sample of this workload's tokens, all host cores."""
+    import oracle
+    cores = os.cpu_count() or 1
+    T = inputs["x"].shape[0]
+    n = min(T, cores)
+    sample = list(range(n))
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.moe_forward(inputs, cfg.k, tokens=sample, threads=n)
+        done += n
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": done / el, "unit": "tokens/s", "cores": n, "kind": "oracle",
+            "sample": f"tokens 0..{n - 1} of the {cfg.name} batch, float64 C oracle with OpenMP over tokens, "
+                      f"repeated for {el:.1f} s ({done} tokens)"}
+
+
+def launches_per_call(T: int, decode: bool) -> int:
+    """Kernels of ours per layer call (memset nodes not counted)."""
+    route = 1 if T <= 64 else 3  # one fused router, or router + scan + scatter
+    if decode:
+        return route + 3  # gate_up GEMV, down GEMV, combine
+    gather = 1 if T <= 64 else 0  # the large-T scatter gathers rows itself
+    return route + gather + 3  # gate_up GEMM, down GEMM, combine
+
+
+def dtype_of(path_decode: bool) -> str:
+    return ("mxfp4 codes -> f16 (exact), f16 x f16 products, fp32 accumulate" if path_decode
+            else "mxfp4 -> bf16 (exact), bf16 tcgen05 MMA, fp32 accumulate")
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    from mxfp4_expert_ffn_bias_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    from mxfp4_expert_ffn_bias_b200 import moe
+
+    peaks, peaks_kind = load_peaks()
+    cfg = CONFIGS[args.config]
+    T = cfg.T
+    inputs = make_inputs(cfg, seed=args.seed)  # same replica on every rank (weak scaling)
+    dev = upload(inputs, torch)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    path = args.path
+    decode = path == 1 or (path == 0 and T <= 64)
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    r = measure(moe, torch, cfg, dev, T, args.steps, args.warmup, path, flush, sampler, args.decode_kernel)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = sum(r["step_ms"])
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = world * T / (ms_step / 1e3)
+
+    bytes_alg, flops_alg = layer_units(cfg, r["n_touched"], T)
+    gu_bytes, gu_flops = gateup_units(cfg, r["n_touched"], T)
+    gu_ms = r["stage_ms"][1]
+    if decode:
+        achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+        kname = "moe::gemv_mma_kernel<true>" if args.decode_kernel == 1 else "moe::gemv_kernel<true>"
+        roof = {"bound": "hbm", "kernel": f"gate_up GEMV ({kname})", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "peak_kind": f"{peaks_kind} HBM copy bandwidth",
+                "algorithmic_bytes_per_launch": gu_bytes}
+    else:
+        achieved = gu_flops / (gu_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM (moe::grouped_mxfp4_gemm<.., true>)",
+                "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                "peak_kind": f"{peaks_kind} dense bf16 (burst)", "algorithmic_flops_per_launch": gu_flops}
+    layer_gbs = bytes_alg / (ms_step / 1e3) / 1e9
+    layer_tflops = flops_alg / (ms_step / 1e3) / 1e12
+    line = {
+        "metric": "MoE-layer tokens/s",
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": dtype_of(decode),
+        "data": "synthetic (seeded generator gen/synth.py, random MXFP4 weights)",
+        "config": {"workload": cfg.name, "T": T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.k,
+                   "path": "decode GEMV" if decode else "grouped tcgen05 GEMM",
+                   "experts_touched": r["n_touched"],
+                   "l2": "flushed before every timed step (256 MiB write, outside the step's events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "layer": {"algorithmic_bytes": bytes_alg, "algorithmic_flops": flops_alg, "GB/s": round(layer_gbs, 1),
+                  "hbm_frac": round(layer_gbs / peaks["hbm_gbs"], 4), "TFLOP/s": round(layer_tflops, 2),
+                  "stage_ms": {n: round(v, 5) for n, v in zip(moe.STAGE_NAMES, r["stage_ms"])}},
+        "gpu_launches": args.steps * (launches_per_call(T, decode)),
+    }
+    line["clocks"] = sampler.summary()
+
+    # end to end through the public API with host buffers
+    e2e_ms, bi, bo = measure_e2e(moe, torch, cfg, dev, inputs["x"], T, args.steps, min(args.warmup, 5), path,
+                                 flush, args.decode_kernel)
+    e2e_step = sum(e2e_ms) / len(e2e_ms)
+    line["e2e"] = {"value": round(world * T / (e2e_step / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": bi,
+                   "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_step, 5),
+                   "api": "moe_forward_hostio (pinned host x/out)"}
+
+    if not args.no_extra and args.config == DEFAULT_CONFIG:
+        pcfg = CONFIGS["gpt-oss-20b-prefill"]
+        pin = make_inputs(pcfg, seed=args.seed)
+        del dev
+        pdev = upload(pin, torch)
+        psteps = max(5, min(args.steps, 20))
+        pr = measure(moe, torch, pcfg, pdev, pcfg.T, psteps, 3, 0, flush)
+        pms = sum(pr["step_ms"]) / psteps
+        pb, pf = layer_units(pcfg, pr["n_touched"], pcfg.T)
+        gb, gf = gateup_units(pcfg, pr["n_touched"], pcfg.T)
+        gms = pr["stage_ms"][1]
+        line["extra"] = {"prefill": {
+            "workload": pcfg.name, "tokens/s": round(pcfg.T / (pms / 1e3), 1), "ms_per_step": round(pms, 4),
+            "layer_TFLOP/s": round(pf / (pms / 1e3) / 1e12, 1),
+            "layer_tensor_frac": round(pf / (pms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "gate_up_TFLOP/s": round(gf / (gms / 1e3) / 1e12, 1),
+            "gate_up_tensor_frac": round(gf / (gms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "stage_ms": {n: round(v, 4) for n, v in zip(moe.STAGE_NAMES, pr["stage_ms"])},
+            "steps": psteps, "peak_kind": f"{peaks_kind} dense bf16 burst {peaks['bf16_tflops']} TFLOP/s"}}
+        del pdev
+
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(cfg, inputs)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    cfg = CONFIGS[args.config]
+    inputs = make_inputs(cfg, seed=args.seed)
+    cores = os.cpu_count() or 1
+    n = min(cfg.T, cores)
+    sample = list(range(n))
+    for _ in range(args.warmup):
+        oracle.moe_forward(inputs, cfg.k, tokens=sample[:1], threads=1)
+    budget = 240.0
+    t0 = time.perf_counter()
+    times = []
+    for i in range(args.steps):
+        s = time.perf_counter()
+        oracle.moe_forward(inputs, cfg.k, tokens=sample, threads=n)
+        times.append(time.perf_counter() - s)
+        if time.perf_counter() - t0 > budget:
+            break
+    el = sum(times)
+    value = len(times) * n / el
+    line = {
+        "impl": "reference", "metric": "MoE-layer tokens/s", "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": len(times), "warmup": args.warmup, "ms_per_step": round(1e3 * el / len(times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generator gen/synth.py)",
+        "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.k,
+                   "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": n, "kind": "oracle",
+                         "sample": f"tokens 0..{n - 1} of the {cfg.name} batch per step (float64 C oracle, "
+                                   f"OpenMP over tokens)"},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    if len(times) < args.steps:
+        line["note"] = f"stopped after {len(times)} of {args.steps} steps at the {budget:.0f} s budget"
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+/*
+ * mxfp4_moe: the GPT-OSS mixture-of-experts feed-forward layer with MXFP4
+ * experts, on one NVIDIA B200 (sm_100a).
+ *
+ * The layer (ZeroModels GPT-OSS docs, GPT-OSS section, the "Mixture-of-experts
+ * feed-forward" and "MXFP4 experts" bullets) computes, per token t:
+ *   logits = x[t] . router_w^T + router_b                          (fp32)
+ *   S      = the top_k largest logits, descending (ties: lower index)
+ *   w      = softmax over the top_k selected logits only
+ *   for each selected expert e:
+ *     h    = x[t] . dequant(gate_up[e])^T + gate_up_bias[e]        [2I]
+ *     gate = h[0::2], up = h[1::2]    (interleaved rows: MaxText PR 2647,
+ *            "1 Support many-to-one transform"; Megatron-Bridge GPT-OSS bridge,
+ *            GPTOSSMLPGateUpProjMapping)
+ *     a    = (clamp(up, -7, 7) + 1) * g * sigmoid(1.702 * g),  g = min(gate, 7)
+ *     y_e  = a . dequant(down[e])^T + down_bias[e]                 [H]
+ *   out[t] = sum over the selected slots s, in slot order, of w_s * y_{e_s}
+ *
+ * MXFP4 tensors: `blocks` uint8 [E, R, C/32, 16] holds two FP4 E2M1 codes per
+ * byte, element 2j of a 32-element block in the LOW nibble of byte j; `scales`
+ * uint8 [E, R, C/32] holds one E8M0 exponent s per block, meaning 2^(s-127).
+ * gate_up is [E, 2I, H] (rows = outputs, gate/up interleaved) and down is
+ * [E, H, I], the MXFP4-dequantised orientation of the Megatron-Bridge GPT-OSS
+ * bridge docs (maybe_modify_loaded_hf_weight). Dequantised values are exact
+ * in bf16 for 2 <= s <= 252; other scale bytes are outside the contract.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named in a function's doc as "device" must be device memory
+ *    of the current CUDA device, owned by the caller, never freed or retained
+ *    by the library beyond the call. bf16 tensors are passed as void* and
+ *    hold raw bf16 bit patterns; all tensors are dense row-major.
+ *  - Device pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). All device
+ *    work is enqueued on it asynchronously; the call returns before it runs
+ *    unless stated otherwise.
+ *  - Every function returns a status code and never throws. Arguments are
+ *    validated on the host before anything is enqueued; on an error nothing
+ *    is enqueued.
+ *  - One handle must not be used by two host threads or two streams at once.
+ */
+#ifndef MXFP4_MOE_H_
+#define MXFP4_MOE_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* null pointer, bad size, misalignment, T > max_T ... */
+  MOE_ERR_UNSUPPORTED = 2,    /* shape outside what the kernels support */
+  MOE_ERR_CUDA = 3,           /* a CUDA runtime/driver call failed (sticky errors included) */
+  MOE_ERR_OOM = 4,            /* workspace allocation failed in moe_create */
+  MOE_ERR_DEVICE_TIMEOUT = 5  /* a bounded device-side wait gave up; see moe_sync_status */
+} moe_status_t;
+
+typedef struct moe_ctx* moe_handle_t;
+
+/* Options for moe_set_option. */
+enum moe_option {
+  MOE_OPT_PATH = 1,          /* 0 = auto, 1 = decode path (routed-expert GEMV), 2 = prefill path
+                                (grouped tcgen05 GEMMs). Default 0. */
+  MOE_OPT_DECODE_MAX_T = 2,  /* auto path uses decode when T <= this. Default 64. */
+  MOE_OPT_SPIN_LIMIT = 3,    /* microseconds a device-side wait may last before the kernel gives up and
+                                reports MOE_ERR_DEVICE_TIMEOUT through moe_sync_status (default 2000000). */
+  MOE_OPT_DECODE_KERNEL = 5, /* decode-path GEMV engine: 0 = CUDA-core mixed-precision FMAs, 1 = m16n8k16
+                                warp MMAs (default). Both compute the same products in fp32. */
+  MOE_OPT_STAGE_EVENTS = 4   /* n > 0: record CUDA events on each call's stream before the first kernel and
+                                after each of the MOE_NUM_STAGES stages, for up to n calls (a ring; read
+                                and reset with moe_stage_times). 0 = off. */
+};
+
+/* Stages timed by MOE_OPT_STAGE_EVENTS: 0 routing (router, top-k, permutation, row gather),
+   1 gate_up (GEMV or grouped GEMM + SwiGLU), 2 down (GEMV or grouped GEMM), 3 combine. */
+#define MOE_NUM_STAGES 4
+
+/*
+ * Create a layer handle for hidden size H, expert width I, E experts and
+ * top_k routed experts per token, for up to max_T tokens per call.
+ * Requires H % 64 == 0, I % 64 == 0, 1 <= top_k <= 8, top_k <= E <= 256,
+ * 1 <= max_T <= 65536. All workspace device memory (sized by max_T) is
+ * allocated here on the current device, so moe_forward never allocates.
+ * On success *out receives the handle; on failure *out is untouched.
+ */
+moe_status_t moe_create(int H, int I, int E, int top_k, int max_T, moe_handle_t* out);
+
+/*
+ * Run the layer on T tokens (1 <= T <= max_T).
+ *   x              device bf16  [T, H]
+ *   router_w       device fp32  [E, H]
+ *   router_b       device fp32  [E]
+ *   gate_up_blocks device uint8 [E, 2I, H/32, 16]
+ *   gate_up_scales device uint8 [E, 2I, H/32]
+ *   gate_up_bias   device bf16  [E, 2I]   (interleaved like the rows)
+ *   down_blocks    device uint8 [E, H, I/32, 16]
+ *   down_scales    device uint8 [E, H, I/32]
+ *   down_bias      device bf16  [E, H]
+ *   out            device bf16  [T, H]   (written; must not alias inputs)
+ * Results are deterministic: the same inputs give the same bits.
+ */
+moe_status_t moe_forward(moe_handle_t h, const void* x, const float* router_w, const float* router_b,
+                         const uint8_t* gate_up_blocks, const uint8_t* gate_up_scales, const void* gate_up_bias,
+                         const uint8_t* down_blocks, const uint8_t* down_scales, const void* down_bias, int T,
+                         void* out, void* stream);
+
+/*
+ * Same as moe_forward, but x and out are HOST pointers (bf16 [T, H] each;
+ * pinned memory gives the best copy speed). The call copies x to the
+ * handle's device staging buffer, runs the layer, copies the result back
+ * and synchronises `stream` before returning, so out is valid on return.
+ * The weight arguments are device pointers as in moe_forward.
+ */
+moe_status_t moe_forward_hostio(moe_handle_t h, const void* x_host, const float* router_w, const float* router_b,
+                                const uint8_t* gate_up_blocks, const uint8_t* gate_up_scales,
+                                const void* gate_up_bias, const uint8_t* down_blocks, const uint8_t* down_scales,
+                                const void* down_bias, int T, void* out_host, void* stream);
+
+/* Free the handle's workspace. Synchronises the device first. NULL is a no-op. */
+moe_status_t moe_destroy(moe_handle_t h);
+
+/* Static, NUL-terminated name of a status code. */
+const char* moe_status_string(moe_status_t s);
+
+/* Set one of enum moe_option. Takes effect on the next call. */
+moe_status_t moe_set_option(moe_handle_t h, int opt, long long value);
+
+/*
+ * Wait for the handle's last stream to finish, then read and clear the
+ * device status word that bounded device-side waits write when they give up.
+ * Returns MOE_ERR_DEVICE_TIMEOUT if one did, MOE_ERR_CUDA on a CUDA error.
+ */
+moe_status_t moe_sync_status(moe_handle_t h);
+
+/*
+ * Device time in milliseconds of each stage, summed over the moe_forward
+ * calls recorded since MOE_OPT_STAGE_EVENTS was set or this function was last
+ * called (at most the ring size; later calls overwrite the oldest). Waits for
+ * those calls' events, writes the sums to ms[0..MOE_NUM_STAGES-1] and the
+ * number of calls to *n_calls, then empties the ring. n >= MOE_NUM_STAGES.
+ */
+moe_status_t moe_stage_times(moe_handle_t h, float* ms, int n, int* n_calls);
+
+/* ---- test hooks: the same device code as the layer's kernels ---- */
+
+/*
+ * Dequantise an MXFP4 tensor [rows, cols] (blocks device uint8
+ * [rows, cols/32, 16], scales device uint8 [rows, cols/32]) to bf16 bit
+ * patterns out_bf16 (device, [rows, cols]) with the device routine the
+ * grouped GEMMs use to fill their shared-memory weight tiles.
+ * cols % 32 == 0; rows, cols >= 1.
+ */
+moe_status_t moe_debug_dequant(const uint8_t* blocks, const uint8_t* scales, int rows, int cols, void* out_bf16,
+                               void* stream);
+
+/*
+ * Convert n packed bytes (device uint8 [n]) to f16x2 pairs (device uint32 [n],
+ * low half = low nibble) with the FP4 converter the decode GEMVs use.
+ */
+moe_status_t moe_debug_decode_codes(const uint8_t* bytes, int n, uint32_t* out_f16x2, void* stream);
+
+/*
+ * Router, top-k, softmax and the counting-sort permutation of a call of T
+ * tokens, exposed for testing. Outputs (device, may be NULL when not wanted):
+ *   idx     int32 [T, top_k]   selected experts, descending logit
+ *   w       fp32  [T, top_k]   softmax over the selected logits
+ *   perm    int32 [T*top_k]    permuted row p -> pair index t*top_k + s,
+ *                              grouped by expert, ascending pair index inside
+ *                              each expert
+ *   offsets int32 [E+1]        start row of each expert's group in perm
+ */
+moe_status_t moe_debug_route(moe_handle_t h, const void* x, const float* router_w, const float* router_b, int T,
+                             int* idx, float* w, int* perm, int* offsets, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXFP4_MOE_H_ */

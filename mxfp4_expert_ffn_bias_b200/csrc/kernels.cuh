@@ -1,0 +1,94 @@
+// Kernel declarations shared between the translation units of the library.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+size_t route_smem_bytes(int E);
+constexpr int kRouteTokPerBlock = 32;  // tokens per large-T router block (= one scatter chunk)
+constexpr int kSmallT = 64;            // calls with T <= kSmallT route in one launch
+
+// Routing results written by the small-T router.
+struct RouteOut {
+  int* idx;
+  float* w;
+  int* counts;
+  int* offsets;
+  int* mt_off;
+  int* perm;
+  int* touched;
+  int* n_touched;
+  int* xexp;
+};
+
+size_t route_small_smem_bytes(int T, int E, int k, int HC);
+__global__ void route_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ rw,
+                                   const float* __restrict__ rb, int T, int H, int E, int k, int HC,
+                                   float* __restrict__ partial, float* __restrict__ pmax, int* __restrict__ ticket,
+                                   RouteOut o);
+__global__ void route_topk_kernel(const uint16_t* __restrict__ x, const float* __restrict__ rw,
+                                  const float* __restrict__ rb, int T, int H, int E, int k, int* __restrict__ idx_out,
+                                  float* __restrict__ w_out, int* __restrict__ counts,
+                                  int* __restrict__ chunk_counts, int* __restrict__ xexp);
+__global__ void route_scan_kernel(const int* __restrict__ counts, const int* __restrict__ chunk_counts, int nchunk,
+                                  int E, int* __restrict__ chunk_base, int* __restrict__ offsets,
+                                  int* __restrict__ mt_off, int* __restrict__ touched, int* __restrict__ n_touched);
+__global__ void route_scatter_kernel(const int* __restrict__ idx, const int* __restrict__ chunk_base, int T, int E,
+                                     int k, const uint16_t* __restrict__ x, int H, int gather,
+                                     int* __restrict__ perm, uint16_t* __restrict__ x_perm);
+__global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ perm, int k, int H,
+                                   uint16_t* __restrict__ x_perm);
+__global__ void combine_kernel(const float* __restrict__ slot, int T, int H, int k, uint16_t* __restrict__ out);
+__global__ void debug_dequant_kernel(const uint8_t* __restrict__ blocks, const uint8_t* __restrict__ scales,
+                                     int rows, int cols, uint16_t* __restrict__ out);
+__global__ void debug_decode_codes_kernel(const uint8_t* __restrict__ bytes, int n, uint32_t* __restrict__ out);
+
+// Decode path (routed-expert GEMVs on the CUDA cores).
+struct GemvArgs {
+  const uint8_t* blocks;   // [E, R, C/32, 16]
+  const uint8_t* scales;   // [E, R, C/32]
+  const uint16_t* bias;    // bf16 [E, R]
+  const int* counts;       // [E]
+  const int* offsets;      // [E+1]
+  const int* touched;      // [E]
+  const int* n_touched;    // [1]
+  const int* perm;         // [T*k]
+  const uint16_t* xin;     // gate_up: bf16 x [T, H]; down: f16 act [T*k, I] (permuted rows)
+  const int* xexp;         // gate_up: [T] per-token exponent (staged tokens are x * 2^-xexp)
+  const float* wroute;     // down: routing weights [T*k]
+  uint16_t* act_out;       // gate_up: f16 act [T*k, I]
+  float* slot_out;         // down: fp32 [T*k, H] by pair index
+  int R, C, k;
+};
+constexpr int kGemvRows = 64;    // weight rows per block
+constexpr int kGemvTok = 8;      // tokens per pass
+size_t gemv_smem_bytes(int C);
+cudaError_t configure_gemv(int Cmax);
+// variant 0: CUDA-core mixed-precision FMAs; 1: m16n8k16 warp MMAs (same numerics)
+cudaError_t launch_gemv_gateup(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st);
+cudaError_t launch_gemv_down(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st);
+
+// Prefill path (grouped tcgen05 GEMMs with in-shared-memory dequantisation).
+struct GemmArgs {
+  const uint8_t* blocks;   // [E, N, K/32, 16]
+  const uint8_t* scales;   // [E, N, K/32]
+  const uint16_t* bias;    // bf16 [E, N]
+  const int* counts;       // [E]
+  const int* offsets;      // [E+1]
+  const int* mt_off;       // [E+1]
+  const int* perm;         // [rows]
+  const float* wroute;     // [T*k] (down)
+  uint16_t* act_out;       // bf16 [rows, N/2] (gate_up)
+  float* slot_out;         // fp32 [T*k, N] (down)
+  unsigned* status;
+  long long spin_limit;
+  int N, K, E, k;
+  int total_rows;          // rows of the A tensor (T*k)
+};
+// Host: build tensor maps and launch. a_ptr is the bf16 A tensor [total_rows, K].
+cudaError_t launch_gemm_gateup(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st);
+cudaError_t launch_gemm_down(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st);
+int gemm_pick_bn(int N);
+
+}  // namespace moe

@@ -1,0 +1,416 @@
+// The C ABI of the library: argument checking, workspace ownership and the
+// launch sequence of one layer call. Nothing here computes the layer; every
+// step runs in the kernels of route.cu, gemv.cu and gemm_sm100.cu.
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_CHECK_CUDA(call)                 \
+  do {                                       \
+    cudaError_t err_ = (call);               \
+    if (err_ != cudaSuccess) return from_cuda(err_); \
+  } while (0)
+
+template <class T>
+cudaError_t alloc(T** p, size_t n) {
+  return cudaMalloc(reinterpret_cast<void**>(p), n * sizeof(T) + 16);
+}
+
+void free_ws(Workspace& w) {
+  void* ptrs[] = {w.counts,  w.offsets, w.mt_off,  w.touched, w.n_touched,    w.idx,        w.w,
+                  w.perm,    w.xexp,    w.x_perm,  w.act,     w.slot,         w.x_stage,    w.out_stage,
+                  w.status,  w.partial, w.pmax,    w.ticket,  w.chunk_counts, w.chunk_base};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  w = Workspace{};
+}
+
+void free_events(moe_ctx* h) {
+  if (h->ev_ring) {
+    for (int i = 0; i < h->ev_slots * (MOE_NUM_STAGES + 1); ++i)
+      if (h->ev_ring[i]) cudaEventDestroy(h->ev_ring[i]);
+    delete[] h->ev_ring;
+  }
+  h->ev_ring = nullptr;
+  h->ev_slots = h->ev_next = h->ev_count = 0;
+}
+
+// Per-kernel attributes (dynamic shared memory limits), set once per handle.
+cudaError_t configure_kernels(const moe_ctx* h) {
+  const int T = h->max_T < kSmallT ? h->max_T : kSmallT;
+  cudaError_t e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)route_small_smem_bytes(T, h->E, h->k, h->HC));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)route_smem_bytes(h->E));
+  if (e != cudaSuccess) return e;
+  return configure_gemv(h->H > h->I ? h->H : h->I);
+}
+
+moe_status_t check_weights(const moe_ctx* h, const void* x, const float* rw, const float* rb, const uint8_t* gub,
+                           const uint8_t* gus, const void* gubias, const uint8_t* db, const uint8_t* ds,
+                           const void* dbias, int T, const void* out) {
+  if (!h || !x || !rw || !rb || !gub || !gus || !gubias || !db || !ds || !dbias || !out) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || T > h->max_T) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, rw, rb, gub, gus, gubias, db, ds, dbias, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+}  // namespace
+
+MOE_API const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_OOM: return "MOE_ERR_OOM";
+    case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+MOE_API moe_status_t moe_create(int H, int I, int E, int top_k, int max_T, moe_handle_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  if (H < 64 || I < 64 || H % 64 || I % 64 || top_k < 1 || top_k > 8 || E < top_k || E > 256 || max_T < 1 ||
+      max_T > 65536)
+    return MOE_ERR_INVALID_ARG;
+  moe_ctx* h = new (std::nothrow) moe_ctx;
+  if (!h) return MOE_ERR_OOM;
+  h->H = H;
+  h->I = I;
+  h->E = E;
+  h->k = top_k;
+  h->max_T = max_T;
+  if (cudaGetDevice(&h->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&h->sm_count, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess) {
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  const size_t Tk = (size_t)max_T * top_k;
+  // small-T router split of H: the largest number of chunks (a divisor of H/64) keeping chunks >= 192 wide
+  h->nHC = 1;
+  for (int n = 1; n <= H / 64; ++n)
+    if ((H / 64) % n == 0 && H / n >= 192) h->nHC = n;
+  h->HC = H / h->nHC;
+  const size_t nchunk = ((size_t)max_T + kRouteTokPerBlock - 1) / kRouteTokPerBlock;
+  Workspace& w = h->ws;
+  bool ok = alloc(&w.counts, E) == cudaSuccess && alloc(&w.offsets, E + 1) == cudaSuccess &&
+            alloc(&w.mt_off, E + 1) == cudaSuccess && alloc(&w.touched, E) == cudaSuccess &&
+            alloc(&w.n_touched, 1) == cudaSuccess && alloc(&w.idx, Tk) == cudaSuccess &&
+            alloc(&w.w, Tk) == cudaSuccess && alloc(&w.perm, Tk) == cudaSuccess &&
+            alloc(&w.xexp, (size_t)max_T) == cudaSuccess && alloc(&w.x_perm, Tk * H) == cudaSuccess &&
+            alloc(&w.act, Tk * I) == cudaSuccess && alloc(&w.slot, Tk * H) == cudaSuccess &&
+            alloc(&w.x_stage, (size_t)max_T * H) == cudaSuccess &&
+            alloc(&w.out_stage, (size_t)max_T * H) == cudaSuccess && alloc(&w.status, 1) == cudaSuccess &&
+            alloc(&w.partial, (size_t)h->nHC * kSmallT * E) == cudaSuccess &&
+            alloc(&w.pmax, (size_t)h->nHC * kSmallT) == cudaSuccess && alloc(&w.ticket, 1) == cudaSuccess &&
+            alloc(&w.chunk_counts, nchunk * E) == cudaSuccess && alloc(&w.chunk_base, nchunk * E) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();  // clear the allocation error
+    free_ws(w);
+    delete h;
+    return MOE_ERR_OOM;
+  }
+  if (cudaMemset(w.status, 0, sizeof(unsigned)) != cudaSuccess || cudaMemset(w.ticket, 0, sizeof(int)) != cudaSuccess ||
+      configure_kernels(h) != cudaSuccess) {
+    free_ws(w);
+    delete h;
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_destroy(moe_handle_t h) {
+  if (!h) return MOE_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  free_ws(h->ws);
+  free_events(h);
+  delete h;
+  return from_cuda(e);
+}
+
+MOE_API moe_status_t moe_set_option(moe_handle_t h, int opt, long long v) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  switch (opt) {
+    case MOE_OPT_PATH:
+      if (v < 0 || v > 2) return MOE_ERR_INVALID_ARG;
+      h->path_opt = (int)v;
+      return MOE_OK;
+    case MOE_OPT_DECODE_MAX_T:
+      if (v < 0 || v > 65536) return MOE_ERR_INVALID_ARG;
+      h->decode_max_T = (int)v;
+      return MOE_OK;
+    case MOE_OPT_SPIN_LIMIT:
+      if (v < 1) return MOE_ERR_INVALID_ARG;
+      h->spin_limit = v;
+      return MOE_OK;
+    case MOE_OPT_DECODE_KERNEL:
+      if (v < 0 || v > 1) return MOE_ERR_INVALID_ARG;
+      h->gemv_variant = (int)v;
+      return MOE_OK;
+    case MOE_OPT_STAGE_EVENTS: {
+      if (v < 0 || v > 100000) return MOE_ERR_INVALID_ARG;
+      if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+      free_events(h);
+      if (v == 0) return MOE_OK;
+      const int n = (int)v * (MOE_NUM_STAGES + 1);
+      h->ev_ring = new (std::nothrow) cudaEvent_t[n]();
+      if (!h->ev_ring) return MOE_ERR_OOM;
+      h->ev_slots = (int)v;
+      for (int i = 0; i < n; ++i)
+        if (cudaEventCreate(&h->ev_ring[i]) != cudaSuccess) {
+          free_events(h);
+          return MOE_ERR_CUDA;
+        }
+      return MOE_OK;
+    }
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+MOE_API moe_status_t moe_sync_status(moe_handle_t h) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  MOE_CHECK_CUDA(cudaStreamSynchronize(h->last_stream));
+  unsigned st = 0;
+  MOE_CHECK_CUDA(cudaMemcpy(&st, h->ws.status, sizeof st, cudaMemcpyDeviceToHost));
+  MOE_CHECK_CUDA(cudaMemset(h->ws.status, 0, sizeof st));
+  return (st & kStatusTimeout) ? MOE_ERR_DEVICE_TIMEOUT : MOE_OK;
+}
+
+namespace {
+
+// Router + top-k + softmax, then the stable counting sort of the (token, slot)
+// pairs by expert; with `gather`, also the expert-grouped copy of x rows.
+moe_status_t enqueue_route(moe_handle_t h, const void* x, const float* rw, const float* rb, int T, bool gather,
+                           cudaStream_t st) {
+  Workspace& w = h->ws;
+  const int Tk = T * h->k, E = h->E, H = h->H, k = h->k;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  if (T <= kSmallT) {
+    RouteOut o{w.idx, w.w, w.counts, w.offsets, w.mt_off, w.perm, w.touched, w.n_touched, w.xexp};
+    dim3 grid((E + 7) / 8, h->nHC);
+    route_small_kernel<<<grid, 256, route_small_smem_bytes(T, E, k, h->HC), st>>>(xb, rw, rb, T, H, E, k, h->HC,
+                                                                                 w.partial, w.pmax, w.ticket, o);
+    MOE_CHECK_CUDA(cudaGetLastError());
+    if (gather) {
+      gather_rows_kernel<<<Tk, 128, 0, st>>>(xb, w.perm, k, H, w.x_perm);
+      MOE_CHECK_CUDA(cudaGetLastError());
+    }
+    return MOE_OK;
+  }
+  const int nchunk = (T + kRouteTokPerBlock - 1) / kRouteTokPerBlock;
+  MOE_CHECK_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(int) * E, st));
+  route_topk_kernel<<<nchunk, 256, route_smem_bytes(E), st>>>(xb, rw, rb, T, H, E, k, w.idx, w.w, w.counts,
+                                                             w.chunk_counts, w.xexp);
+  MOE_CHECK_CUDA(cudaGetLastError());
+  route_scan_kernel<<<E, 256, 0, st>>>(w.counts, w.chunk_counts, nchunk, E, w.chunk_base, w.offsets, w.mt_off,
+                                       w.touched, w.n_touched);
+  MOE_CHECK_CUDA(cudaGetLastError());
+  route_scatter_kernel<<<nchunk, 256, 0, st>>>(w.idx, w.chunk_base, T, E, k, xb, H, gather ? 1 : 0, w.perm,
+                                               w.x_perm);
+  MOE_CHECK_CUDA(cudaGetLastError());
+  return MOE_OK;
+}
+
+bool use_decode(const moe_ctx* h, int T) {
+  if (h->path_opt == 1) return true;
+  if (h->path_opt == 2) return false;
+  return T <= h->decode_max_T;
+}
+
+moe_status_t enqueue_forward(moe_handle_t h, const void* x, const float* rw, const float* rb, const uint8_t* gub,
+                             const uint8_t* gus, const void* gubias, const uint8_t* db, const uint8_t* ds,
+                             const void* dbias, int T, void* out, cudaStream_t st) {
+  Workspace& w = h->ws;
+  const int H = h->H, I = h->I, E = h->E, k = h->k, Tk = T * k;
+  const bool rec = h->ev_slots > 0;
+  cudaEvent_t* ev = rec ? h->ev_ring + (size_t)h->ev_next * (MOE_NUM_STAGES + 1) : nullptr;
+  if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[0], st));
+  const bool decode = use_decode(h, T);
+  moe_status_t s = enqueue_route(h, x, rw, rb, T, !decode, st);
+  if (s != MOE_OK) return s;
+  if (decode) {
+    if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[1], st));
+    const int max_touched = Tk < E ? Tk : E;
+    GemvArgs g{};
+    g.counts = w.counts;
+    g.offsets = w.offsets;
+    g.touched = w.touched;
+    g.n_touched = w.n_touched;
+    g.perm = w.perm;
+    g.k = k;
+    g.blocks = gub;
+    g.scales = gus;
+    g.bias = static_cast<const uint16_t*>(gubias);
+    g.xin = static_cast<const uint16_t*>(x);
+    g.xexp = w.xexp;
+    g.act_out = w.act;
+    g.R = 2 * I;
+    g.C = H;
+    MOE_CHECK_CUDA(launch_gemv_gateup(g, max_touched, h->gemv_variant, h->sm_count, st));
+    if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[2], st));
+    g.blocks = db;
+    g.scales = ds;
+    g.bias = static_cast<const uint16_t*>(dbias);
+    g.xin = w.act;
+    g.xexp = nullptr;
+    g.wroute = w.w;
+    g.slot_out = w.slot;
+    g.act_out = nullptr;
+    g.R = H;
+    g.C = I;
+    MOE_CHECK_CUDA(launch_gemv_down(g, max_touched, h->gemv_variant, h->sm_count, st));
+  } else {
+    if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[1], st));
+    GemmArgs g{};
+    g.counts = w.counts;
+    g.offsets = w.offsets;
+    g.mt_off = w.mt_off;
+    g.perm = w.perm;
+    g.status = w.status;
+    g.spin_limit = h->spin_limit;
+    g.E = E;
+    g.k = k;
+    g.total_rows = Tk;
+    g.blocks = gub;
+    g.scales = gus;
+    g.bias = static_cast<const uint16_t*>(gubias);
+    g.act_out = w.act;
+    g.N = 2 * I;
+    g.K = H;
+    MOE_CHECK_CUDA(launch_gemm_gateup(g, w.x_perm, h->sm_count, st));
+    if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[2], st));
+    g.blocks = db;
+    g.scales = ds;
+    g.bias = static_cast<const uint16_t*>(dbias);
+    g.act_out = nullptr;
+    g.wroute = w.w;
+    g.slot_out = w.slot;
+    g.N = H;
+    g.K = I;
+    MOE_CHECK_CUDA(launch_gemm_down(g, w.act, h->sm_count, st));
+  }
+  if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[3], st));
+  const int threads = 256;
+  long long n4 = (long long)T * H / 4;
+  int blocks = (int)((n4 + threads - 1) / threads);
+  const int cap = h->sm_count * 8;
+  if (blocks > cap) blocks = cap;
+  combine_kernel<<<blocks, threads, 0, st>>>(w.slot, T, H, k, static_cast<uint16_t*>(out));
+  MOE_CHECK_CUDA(cudaGetLastError());
+  if (rec) {
+    MOE_CHECK_CUDA(cudaEventRecord(ev[4], st));
+    h->ev_next = (h->ev_next + 1) % h->ev_slots;
+    if (h->ev_count < h->ev_slots) ++h->ev_count;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+MOE_API moe_status_t moe_forward(moe_handle_t h, const void* x, const float* router_w, const float* router_b,
+                                 const uint8_t* gate_up_blocks, const uint8_t* gate_up_scales,
+                                 const void* gate_up_bias, const uint8_t* down_blocks, const uint8_t* down_scales,
+                                 const void* down_bias, int T, void* out, void* stream) {
+  moe_status_t s = check_weights(h, x, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias,
+                                 down_blocks, down_scales, down_bias, T, out);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  return enqueue_forward(h, x, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks,
+                         down_scales, down_bias, T, out, st);
+}
+
+MOE_API moe_status_t moe_forward_hostio(moe_handle_t h, const void* x_host, const float* router_w,
+                                        const float* router_b, const uint8_t* gate_up_blocks,
+                                        const uint8_t* gate_up_scales, const void* gate_up_bias,
+                                        const uint8_t* down_blocks, const uint8_t* down_scales,
+                                        const void* down_bias, int T, void* out_host, void* stream) {
+  if (!h || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  moe_status_t s = check_weights(h, h->ws.x_stage, router_w, router_b, gate_up_blocks, gate_up_scales,
+                                 gate_up_bias, down_blocks, down_scales, down_bias, T, h->ws.out_stage);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  const size_t bytes = (size_t)T * h->H * sizeof(uint16_t);
+  MOE_CHECK_CUDA(cudaMemcpyAsync(h->ws.x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
+  s = enqueue_forward(h, h->ws.x_stage, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias,
+                      down_blocks, down_scales, down_bias, T, h->ws.out_stage, st);
+  if (s != MOE_OK) return s;
+  MOE_CHECK_CUDA(cudaMemcpyAsync(out_host, h->ws.out_stage, bytes, cudaMemcpyDeviceToHost, st));
+  MOE_CHECK_CUDA(cudaStreamSynchronize(st));
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_stage_times(moe_handle_t h, float* ms, int n, int* n_calls) {
+  if (!h || !ms || !n_calls || n < MOE_NUM_STAGES) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < MOE_NUM_STAGES; ++i) ms[i] = 0.f;
+  *n_calls = 0;
+  if (h->ev_slots == 0) return MOE_ERR_INVALID_ARG;
+  const int first = (h->ev_next - h->ev_count + h->ev_slots) % h->ev_slots;
+  for (int c = 0; c < h->ev_count; ++c) {
+    cudaEvent_t* ev = h->ev_ring + (size_t)((first + c) % h->ev_slots) * (MOE_NUM_STAGES + 1);
+    MOE_CHECK_CUDA(cudaEventSynchronize(ev[MOE_NUM_STAGES]));
+    for (int i = 0; i < MOE_NUM_STAGES; ++i) {
+      float t = 0.f;
+      MOE_CHECK_CUDA(cudaEventElapsedTime(&t, ev[i], ev[i + 1]));
+      ms[i] += t;
+    }
+  }
+  *n_calls = h->ev_count;
+  h->ev_count = 0;
+  return MOE_OK;
+}
+
+MOE_API moe_status_t moe_debug_dequant(const uint8_t* blocks, const uint8_t* scales, int rows, int cols,
+                                       void* out_bf16, void* stream) {
+  if (!blocks || !scales || !out_bf16 || rows < 1 || cols < 32 || cols % 32) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(blocks) || !aligned16(out_bf16)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long chunks = (long long)rows * cols / 8;
+  int grid = (int)((chunks + 255) / 256);
+  if (grid > 65535) grid = 65535;
+  debug_dequant_kernel<<<grid, 256, 0, st>>>(blocks, scales, rows, cols, static_cast<uint16_t*>(out_bf16));
+  return from_cuda(cudaGetLastError());
+}
+
+MOE_API moe_status_t moe_debug_decode_codes(const uint8_t* bytes, int n, uint32_t* out, void* stream) {
+  if (!bytes || !out || n < 1) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n % 4 || !aligned16(bytes)) return MOE_ERR_INVALID_ARG;
+  debug_decode_codes_kernel<<<(n / 4 + 255) / 256, 256, 0, st>>>(bytes, n, out);
+  return from_cuda(cudaGetLastError());
+}
+
+MOE_API moe_status_t moe_debug_route(moe_handle_t h, const void* x, const float* rw, const float* rb, int T,
+                                     int* idx, float* w, int* perm, int* offsets, void* stream) {
+  if (!h || !x || !rw || !rb || T < 1 || T > h->max_T) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(rw)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  moe_status_t s = enqueue_route(h, x, rw, rb, T, false, st);
+  if (s != MOE_OK) return s;
+  const size_t Tk = (size_t)T * h->k;
+  if (idx) MOE_CHECK_CUDA(cudaMemcpyAsync(idx, h->ws.idx, Tk * sizeof(int), cudaMemcpyDeviceToDevice, st));
+  if (w) MOE_CHECK_CUDA(cudaMemcpyAsync(w, h->ws.w, Tk * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  if (perm) MOE_CHECK_CUDA(cudaMemcpyAsync(perm, h->ws.perm, Tk * sizeof(int), cudaMemcpyDeviceToDevice, st));
+  if (offsets)
+    MOE_CHECK_CUDA(
+        cudaMemcpyAsync(offsets, h->ws.offsets, (h->E + 1) * sizeof(int), cudaMemcpyDeviceToDevice, st));
+  return MOE_OK;
+}

@@ -1,0 +1,503 @@
+// Router (logits + top-k + softmax over k), the deterministic counting-sort
+// permutation of (token, slot) pairs by expert, the row gather for the grouped
+// GEMMs, the fixed-order slot combine, and two test-hook kernels.
+#include "common.cuh"
+#include "kernels.cuh"
+#include "mx_dequant.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------- router
+
+constexpr int kRouteWarps = 8;
+constexpr int kRouteTokPerWarp = 4;
+constexpr int kRouteTok = kRouteWarps * kRouteTokPerWarp;  // tokens per block (== kRouteTokPerBlock)
+constexpr int kRouteHC = 64;                               // hidden columns per staged chunk
+constexpr int kMaxEJ = 8;                                  // experts per lane (E <= 256)
+static_assert(kRouteTok == kRouteTokPerBlock, "router chunk size");
+
+size_t route_smem_bytes(int E) {
+  return sizeof(float) * ((size_t)kRouteTok * kRouteHC + (size_t)E * (kRouteHC + 1)) + sizeof(int) * 256;
+}
+
+// k rounds of a warp-wide arg-max over the logits lg[j] of experts lane + 32j
+// (ties: lower expert index). Every lane ends with the same sele/selv.
+__device__ __forceinline__ void warp_topk(const float (&lg)[kMaxEJ], int EJ, int E, int k, int* sele, float* selv) {
+  const int lane = threadIdx.x & 31;
+  unsigned taken = 0;
+  for (int s = 0; s < k; ++s) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < kMaxEJ; ++j) {
+      const int e = lane + 32 * j;
+      if (j < EJ && e < E && !(taken & (1u << j)) && (lg[j] > bv || (lg[j] == bv && e < be))) {
+        bv = lg[j];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    selv[s] = bv;
+    sele[s] = be;
+  }
+}
+
+// Softmax over the k selected logits (fp32, max subtracted), as the weights w_s.
+__device__ __forceinline__ void softmax_k(const float* selv, int k, float* w) {
+  float z = 0.f;
+  for (int s = 0; s < k; ++s) {
+    w[s] = expf(selv[s] - selv[0]);
+    z += w[s];
+  }
+  for (int s = 0; s < k; ++s) w[s] /= z;
+}
+
+// Exponent c_t with max|x_t| * 2^-c_t in [2^14, 2^15) (0 for an all-zero row).
+__device__ __forceinline__ int token_exponent(float amax) {
+  int c = 0;
+  if (amax > 0.f) c = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 - 14;
+  return max(-100, min(100, c));
+}
+
+// Large-T router: one block handles 32 tokens against all E experts. Logits
+// are fp32 sums over h in increasing order; lane L of a warp owns experts L,
+// L+32, ... The block also counts its own (token, slot) pairs per expert
+// (chunk_counts[block][e]) for the stable scatter that follows.
+__global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ rw, const float* __restrict__ rb, int T, int H,
+    int E, int k, int* __restrict__ idx_out, float* __restrict__ w_out, int* __restrict__ counts,
+    int* __restrict__ chunk_counts, int* __restrict__ xexp) {
+  extern __shared__ float smem[];
+  float* xs = smem;                               // [kRouteTok][kRouteHC]
+  float* ws = smem + kRouteTok * kRouteHC;        // [E][kRouteHC + 1]
+  int* s_cc = reinterpret_cast<int*>(ws + E * (kRouteHC + 1));  // [E]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * kRouteTok;
+  const int EJ = (E + 31) / 32;
+  for (int e = tid; e < E; e += blockDim.x) s_cc[e] = 0;
+
+  float acc[kRouteTokPerWarp][kMaxEJ];
+#pragma unroll
+  for (int i = 0; i < kRouteTokPerWarp; ++i)
+#pragma unroll
+    for (int j = 0; j < kMaxEJ; ++j) acc[i][j] = 0.f;
+  float amax[kRouteTokPerWarp];
+#pragma unroll
+  for (int i = 0; i < kRouteTokPerWarp; ++i) amax[i] = 0.f;
+
+  for (int h0 = 0; h0 < H; h0 += kRouteHC) {
+    for (int i = tid; i < kRouteTok * kRouteHC / 2; i += blockDim.x) {
+      const int tt = i / (kRouteHC / 2), hh = 2 * (i % (kRouteHC / 2));
+      const int t = t0 + tt;
+      uint32_t v = 0;
+      if (t < T) v = *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + hh);
+      xs[tt * kRouteHC + hh] = bf16_bits_to_float(v & 0xFFFF);
+      xs[tt * kRouteHC + hh + 1] = bf16_bits_to_float(v >> 16);
+    }
+    for (int i = tid; i < E * kRouteHC / 4; i += blockDim.x) {
+      const int e = i / (kRouteHC / 4), hh = 4 * (i % (kRouteHC / 4));
+      const float4 v = *reinterpret_cast<const float4*>(rw + (size_t)e * H + h0 + hh);
+      float* d = ws + e * (kRouteHC + 1) + hh;
+      d[0] = v.x;
+      d[1] = v.y;
+      d[2] = v.z;
+      d[3] = v.w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kRouteTokPerWarp; ++i) {
+      const float* xr = xs + (warp * kRouteTokPerWarp + i) * kRouteHC;
+      amax[i] = fmaxf(amax[i], fmaxf(fabsf(xr[lane]), fabsf(xr[lane + 32])));
+    }
+#pragma unroll 4
+    for (int hh = 0; hh < kRouteHC; ++hh) {
+      float xv[kRouteTokPerWarp];
+#pragma unroll
+      for (int i = 0; i < kRouteTokPerWarp; ++i) xv[i] = xs[(warp * kRouteTokPerWarp + i) * kRouteHC + hh];
+#pragma unroll
+      for (int j = 0; j < kMaxEJ; ++j) {
+        if (j < EJ) {
+          const int e = lane + 32 * j;
+          const float wv = (e < E) ? ws[e * (kRouteHC + 1) + hh] : 0.f;
+#pragma unroll
+          for (int i = 0; i < kRouteTokPerWarp; ++i) acc[i][j] = fmaf(xv[i], wv, acc[i][j]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int i = 0; i < kRouteTokPerWarp; ++i) {
+    const int t = t0 + warp * kRouteTokPerWarp + i;
+    if (t >= T) continue;  // warp-uniform
+    float m = amax[i];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float lg[kMaxEJ];
+#pragma unroll
+    for (int j = 0; j < kMaxEJ; ++j) {
+      const int e = lane + 32 * j;
+      lg[j] = (j < EJ && e < E) ? acc[i][j] + rb[e] : -INFINITY;
+    }
+    int sele[8];
+    float selv[8], w[8];
+    warp_topk(lg, EJ, E, k, sele, selv);
+    if (lane == 0) {
+      softmax_k(selv, k, w);
+      for (int s = 0; s < k; ++s) {
+        idx_out[t * k + s] = sele[s];
+        w_out[t * k + s] = w[s];
+        atomicAdd(&counts[sele[s]], 1);  // integer counts: the same whatever the order
+        atomicAdd(&s_cc[sele[s]], 1);
+      }
+      xexp[t] = token_exponent(m);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) chunk_counts[(size_t)blockIdx.x * E + e] = s_cc[e];
+}
+
+// ---------------------------------------------------------------- stable counting sort (large T)
+
+// Block-wide exclusive prefix over counts[0..E) (E <= 256) into s_off[0..E],
+// and over ceil(counts/kBM) into s_mt[0..E]. Uses warp 0.
+__device__ __forceinline__ void prefix_counts(const int* counts, int E, int* s_off, int* s_mt) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    int c[8], m[8], sc = 0, sm = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      c[j] = (e < E) ? counts[e] : 0;
+      m[j] = (c[j] + kBM - 1) / kBM;
+      sc += c[j];
+      sm += m[j];
+    }
+    int ic = sc, im = sm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, ic, o), b = __shfl_up_sync(0xffffffffu, im, o);
+      if (lane >= o) {
+        ic += a;
+        im += b;
+      }
+    }
+    int ec = ic - sc, em = im - sm;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane * 8 + j;
+      if (e < E) {
+        s_off[e] = ec;
+        s_mt[e] = em;
+      }
+      ec += c[j];
+      em += m[j];
+    }
+    if (lane == 31) {  // totals
+      s_off[E] = ic;
+      s_mt[E] = im;
+    }
+  }
+}
+
+// One block per expert e: exclusive prefix of chunk_counts[:, e] over the
+// router chunks, plus the expert's start row, gives chunk_base[chunk][e]: the
+// first permuted row of chunk's pairs routed to e. Block 0 also publishes
+// offsets, mt_off and the list of touched experts.
+__global__ void __launch_bounds__(256) route_scan_kernel(const int* __restrict__ counts,
+                                                         const int* __restrict__ chunk_counts, int nchunk, int E,
+                                                         int* __restrict__ chunk_base, int* __restrict__ offsets,
+                                                         int* __restrict__ mt_off, int* __restrict__ touched,
+                                                         int* __restrict__ n_touched) {
+  __shared__ int s_off[257], s_mt[257], s_part[256];
+  const int e = blockIdx.x, tid = threadIdx.x;
+  prefix_counts(counts, E, s_off, s_mt);
+  __syncthreads();
+  if (e == 0) {
+    for (int i = tid; i <= E; i += blockDim.x) {
+      offsets[i] = s_off[i];
+      mt_off[i] = s_mt[i];
+    }
+    if (tid == 0) {
+      int n = 0;
+      for (int j = 0; j < E; ++j)
+        if (s_off[j + 1] > s_off[j]) touched[n++] = j;
+      *n_touched = n;
+    }
+  }
+  // each thread owns a contiguous run of chunks
+  const int per = (nchunk + blockDim.x - 1) / blockDim.x;
+  const int c0 = tid * per, c1 = min(nchunk, c0 + per);
+  int sum = 0;
+  for (int c = c0; c < c1; ++c) sum += chunk_counts[(size_t)c * E + e];
+  s_part[tid] = sum;
+  __syncthreads();
+  if (tid < 32) {  // exclusive scan of the 256 partial sums by warp 0
+    int v[8], tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      v[j] = s_part[tid * 8 + j];
+      tot += v[j];
+    }
+    int inc = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, inc, o);
+      if (tid >= o) inc += a;
+    }
+    int run = inc - tot;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int x = v[j];
+      s_part[tid * 8 + j] = run;
+      run += x;
+    }
+  }
+  __syncthreads();
+  int run = s_off[e] + s_part[tid];
+  for (int c = c0; c < c1; ++c) {
+    chunk_base[(size_t)c * E + e] = run;
+    run += chunk_counts[(size_t)c * E + e];
+  }
+}
+
+// One block per router chunk (32 tokens): the stable rank of each pair among
+// the chunk's pairs with the same expert, plus chunk_base, is its permuted row.
+// Optionally copies the token's x row there (the A operand of the gate_up GEMM).
+__global__ void __launch_bounds__(256) route_scatter_kernel(const int* __restrict__ idx,
+                                                            const int* __restrict__ chunk_base, int T, int E, int k,
+                                                            const uint16_t* __restrict__ x, int H, int gather,
+                                                            int* __restrict__ perm, uint16_t* __restrict__ x_perm) {
+  __shared__ int s_idx[kRouteTok * 8], s_dest[kRouteTok * 8];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int t0 = b * kRouteTok;
+  const int P = min(kRouteTok, T - t0) * k;
+  const int p0 = t0 * k;
+  for (int i = tid; i < P; i += blockDim.x) s_idx[i] = idx[p0 + i];
+  __syncthreads();
+  for (int i = tid; i < P; i += blockDim.x) {
+    const int e = s_idx[i];
+    int rank = 0;
+    for (int j = 0; j < i; ++j) rank += (s_idx[j] == e);
+    const int dest = chunk_base[(size_t)b * E + e] + rank;
+    perm[dest] = p0 + i;
+    s_dest[i] = dest;
+  }
+  if (!gather) return;
+  __syncthreads();
+  const int nv = H / 8;
+#pragma unroll 4
+  for (int wi = tid; wi < P * nv; wi += blockDim.x) {
+    const int i = wi / nv, v = wi - i * nv;
+    reinterpret_cast<uint4*>(x_perm + (size_t)s_dest[i] * H)[v] =
+        reinterpret_cast<const uint4*>(x + (size_t)((p0 + i) / k) * H)[v];
+  }
+}
+
+// ---------------------------------------------------------------- small-T router (one launch)
+
+// For T <= kSmallT. Block (eg, hc) computes partial logits of experts
+// [8*eg, 8*eg+8) over hidden columns [hc*HC, (hc+1)*HC) for every token, and
+// (eg == 0) the partial max|x| of each token. The last block to finish (a
+// ticket counter) sums the partials in hc order, runs top-k and softmax for
+// every token, and performs the stable counting sort of all pairs in shared
+// memory; it then re-arms the ticket. The result does not depend on which
+// block finishes last.
+size_t route_small_smem_bytes(int T, int E, int k, int HC) {
+  const size_t a = ((size_t)T * (HC + 2) * 2 + 15) / 16 * 16 + (size_t)8 * (HC + 1) * 4;
+  const size_t b = (size_t)T * E * 4 + (size_t)T * k * 4 + 3 * 260 * 4;
+  return a > b ? a : b;
+}
+
+__global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __restrict__ x,
+                                                          const float* __restrict__ rw,
+                                                          const float* __restrict__ rb, int T, int H, int E, int k,
+                                                          int HC, float* __restrict__ partial,
+                                                          float* __restrict__ pmax, int* __restrict__ ticket,
+                                                          RouteOut o) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int s_last;
+  const int eg = blockIdx.x, hc = blockIdx.y, nHC = gridDim.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h0 = hc * HC;
+  const int XS = HC + 2, WS = HC + 1;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(sm);
+  float* ws = reinterpret_cast<float*>(sm + ((size_t)T * XS * 2 + 15) / 16 * 16);
+  for (int i = tid; i < T * (HC / 2); i += blockDim.x) {
+    const int t = i / (HC / 2), c2 = i % (HC / 2);
+    *reinterpret_cast<uint32_t*>(xs + t * XS + 2 * c2) =
+        *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + 2 * c2);
+  }
+  for (int i = tid; i < 8 * HC; i += blockDim.x) {
+    const int el = i / HC, c = i % HC, e = eg * 8 + el;
+    ws[el * WS + c] = (e < E) ? rw[(size_t)e * H + h0 + c] : 0.f;
+  }
+  __syncthreads();
+  for (int oi = tid; oi < T * 8; oi += blockDim.x) {
+    const int t = oi >> 3, el = oi & 7, e = eg * 8 + el;
+    if (e >= E) continue;
+    const uint16_t* xr = xs + t * XS;
+    const float* wr = ws + el * WS;
+    float acc = 0.f;
+    for (int c = 0; c < HC; ++c) acc = fmaf(bf16_bits_to_float(xr[c]), wr[c], acc);
+    partial[((size_t)hc * T + t) * E + e] = acc;
+  }
+  if (eg == 0) {
+    for (int t = warp; t < T; t += 8) {
+      float m = 0.f;
+      for (int c = lane; c < HC; c += 32) m = fmaxf(m, fabsf(bf16_bits_to_float(xs[t * XS + c])));
+#pragma unroll
+      for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (lane == 0) pmax[(size_t)hc * T + t] = m;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // ---- last block: logits, top-k, softmax, counting sort
+  float* lg = reinterpret_cast<float*>(sm);     // [T][E]
+  int* s_idx = reinterpret_cast<int*>(lg + (size_t)T * E);  // [T*k]
+  int* s_cnt = s_idx + T * k;                   // [E]
+  int* s_off = s_cnt + 260;                     // [E+1]
+  int* s_mt = s_off + 260;                      // [E+1]
+  for (int i = tid; i < T * E; i += blockDim.x) {
+    const int t = i / E, e = i % E;
+    float v = 0.f;
+    for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
+    lg[i] = v + rb[e];
+  }
+  __syncthreads();
+  const int EJ = (E + 31) / 32;
+  for (int t = warp; t < T; t += 8) {
+    float l[kMaxEJ];
+#pragma unroll
+    for (int j = 0; j < kMaxEJ; ++j) {
+      const int e = lane + 32 * j;
+      l[j] = (j < EJ && e < E) ? lg[t * E + e] : -INFINITY;
+    }
+    int sele[8];
+    float selv[8], w[8];
+    warp_topk(l, EJ, E, k, sele, selv);
+    if (lane == 0) {
+      softmax_k(selv, k, w);
+      float m = 0.f;
+      for (int h = 0; h < nHC; ++h) m = fmaxf(m, __ldcg(&pmax[(size_t)h * T + t]));
+      o.xexp[t] = token_exponent(m);
+      for (int s = 0; s < k; ++s) {
+        o.idx[t * k + s] = sele[s];
+        o.w[t * k + s] = w[s];
+        s_idx[t * k + s] = sele[s];
+      }
+    }
+  }
+  __syncthreads();
+  const int Tk = T * k;
+  for (int e = tid; e < E; e += blockDim.x) {
+    int c = 0;
+    for (int p = 0; p < Tk; ++p) c += (s_idx[p] == e);
+    s_cnt[e] = c;
+    o.counts[e] = c;
+  }
+  __syncthreads();
+  prefix_counts(s_cnt, E, s_off, s_mt);
+  __syncthreads();
+  for (int i = tid; i <= E; i += blockDim.x) {
+    o.offsets[i] = s_off[i];
+    o.mt_off[i] = s_mt[i];
+  }
+  if (tid == 0) {
+    int n = 0;
+    for (int j = 0; j < E; ++j)
+      if (s_cnt[j] > 0) o.touched[n++] = j;
+    *o.n_touched = n;
+    *ticket = 0;  // re-arm for the next call
+  }
+  for (int p = tid; p < Tk; p += blockDim.x) {
+    const int e = s_idx[p];
+    int rank = 0;
+    for (int j = 0; j < p; ++j) rank += (s_idx[j] == e);
+    o.perm[s_off[e] + rank] = p;
+  }
+}
+
+// x_perm[p] = x[perm[p] / k]: one block per permuted row, 16-byte vectors.
+__global__ void __launch_bounds__(128) gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ perm,
+                                                          int k, int H, uint16_t* __restrict__ x_perm) {
+  const int p = blockIdx.x;
+  const int t = perm[p] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+  uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)p * H);
+  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) dst[i] = src[i];
+}
+
+// out[t, j] = bf16( sum_{s=0..k-1} slot[t*k+s, j] ), summed in slot order.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ slot, int T, int H, int k,
+                                                      uint16_t* __restrict__ out) {
+  const int H4 = H / 4;
+  const long long n = (long long)T * H4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long t = i / H4;
+    const int j4 = (int)(i % H4);
+    const float4* src = reinterpret_cast<const float4*>(slot + (size_t)t * k * H) + j4;
+    float4 a = src[0];
+    for (int s = 1; s < k; ++s) {
+      const float4 b = src[(size_t)s * H4];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(a.x, a.y);
+    o.y = pack_bf16x2(a.z, a.w);
+    reinterpret_cast<uint2*>(out + (size_t)t * H)[j4] = o;
+  }
+}
+
+// ---------------------------------------------------------------- test hooks
+
+__global__ void debug_dequant_kernel(const uint8_t* __restrict__ blocks, const uint8_t* __restrict__ scales,
+                                     int rows, int cols, uint16_t* __restrict__ out) {
+  const int nb = cols / 32;
+  const long long chunks = (long long)rows * cols / 8;
+  for (long long c = blockIdx.x * (long long)blockDim.x + threadIdx.x; c < chunks;
+       c += (long long)gridDim.x * blockDim.x) {
+    const long long r = c / (cols / 8);
+    const int cc = (int)(c % (cols / 8));  // 8-element chunk within the row
+    const int b = cc / 4;
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(blocks + ((size_t)r * nb + b) * 16 + (cc % 4) * 4);
+    const uint32_t s = scales[(size_t)r * nb + b];
+    *reinterpret_cast<uint4*>(out + (size_t)r * cols + cc * 8) = mx_dequant8_bf16(w, s);
+  }
+}
+
+__global__ void debug_decode_codes_kernel(const uint8_t* __restrict__ bytes, int n, uint32_t* __restrict__ out) {
+  // one 32-bit word (4 packed bytes) per thread, exactly as the decode GEMVs consume them
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (4 * i >= n) return;
+  const uint32_t w = reinterpret_cast<const uint32_t*>(bytes)[i];
+  uint32_t h0, h1, h2, h3;
+  e2m1x8_to_f16x2(w, h0, h1, h2, h3);
+  out[4 * i + 0] = h0;
+  out[4 * i + 1] = h1;
+  out[4 * i + 2] = h2;
+  out[4 * i + 3] = h3;
+}
+
+}  // namespace moe

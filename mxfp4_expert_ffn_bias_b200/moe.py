@@ -1,0 +1,185 @@
+"""Thin ctypes binding of the C ABI in ``include/moe.h``.
+
+Argument marshalling only: every step of the layer runs in the sm_100a
+kernels of ``libmoe_b200.so``. Tensors are torch CUDA tensors (bf16 data may
+be torch.bfloat16 or raw uint16/int16 bit patterns); the current torch CUDA
+stream is passed unless one is given. There is no CPU fallback: if the
+library is missing or fails to load, importing this module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with mxfp4_expert_ffn_bias_b200/build.py "
+                      "(or __graft_entry__.build())")
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED = 2
+MOE_ERR_CUDA = 3
+MOE_ERR_OOM = 4
+MOE_ERR_DEVICE_TIMEOUT = 5
+
+MOE_OPT_PATH = 1
+MOE_OPT_DECODE_MAX_T = 2
+MOE_OPT_SPIN_LIMIT = 3
+MOE_OPT_STAGE_EVENTS = 4
+MOE_OPT_DECODE_KERNEL = 5
+MOE_NUM_STAGES = 4
+STAGE_NAMES = ("route", "gate_up", "down", "combine")
+
+PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+
+# Every symbol the header declares, with its ctypes signature.
+SIGNATURES = {
+    "moe_create": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_P)]),
+    "moe_forward": (_I, [_P] * 10 + [_I, _P, _P]),
+    "moe_forward_hostio": (_I, [_P] * 10 + [_I, _P, _P]),
+    "moe_destroy": (_I, [_P]),
+    "moe_status_string": (ctypes.c_char_p, [_I]),
+    "moe_set_option": (_I, [_P, _I, ctypes.c_longlong]),
+    "moe_sync_status": (_I, [_P]),
+    "moe_stage_times": (_I, [_P, ctypes.POINTER(ctypes.c_float), _I, ctypes.POINTER(_I)]),
+    "moe_debug_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
+    "moe_debug_decode_codes": (_I, [_P, _I, _P, _P]),
+    "moe_debug_route": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
+}
+for _name, (_res, _args) in SIGNATURES.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)}")
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def moe_create(H: int, I: int, E: int, top_k: int, max_T: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_lib.moe_create(H, I, E, top_k, max_T, ctypes.byref(h)), "moe_create")
+    return h
+
+
+def moe_destroy(h) -> None:
+    _check(_lib.moe_destroy(h), "moe_destroy")
+
+
+def moe_set_option(h, opt: int, value: int) -> None:
+    _check(_lib.moe_set_option(h, int(opt), int(value)), "moe_set_option")
+
+
+def moe_sync_status(h) -> int:
+    return int(_lib.moe_sync_status(h))
+
+
+def moe_stage_times(h):
+    """(per-stage device ms summed over the recorded calls, number of calls); empties the ring."""
+    arr = (ctypes.c_float * MOE_NUM_STAGES)()
+    n = ctypes.c_int(0)
+    _check(_lib.moe_stage_times(h, arr, MOE_NUM_STAGES, ctypes.byref(n)), "moe_stage_times")
+    return list(arr), n.value
+
+
+def moe_forward(h, x, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks, down_scales,
+                down_bias, T: int, out, stream=None) -> None:
+    _check(_lib.moe_forward(h, _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(gate_up_blocks), _ptr(gate_up_scales),
+                            _ptr(gate_up_bias), _ptr(down_blocks), _ptr(down_scales), _ptr(down_bias), int(T),
+                            _ptr(out), _stream(stream)), "moe_forward")
+
+
+def moe_forward_hostio(h, x_host: torch.Tensor, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias,
+                       down_blocks, down_scales, down_bias, T: int, out_host: torch.Tensor, stream=None) -> None:
+    if x_host.is_cuda or out_host.is_cuda:
+        raise ValueError("moe_forward_hostio takes host tensors for x and out")
+    _check(_lib.moe_forward_hostio(h, ctypes.c_void_p(x_host.data_ptr()), _ptr(router_w), _ptr(router_b),
+                                   _ptr(gate_up_blocks), _ptr(gate_up_scales), _ptr(gate_up_bias),
+                                   _ptr(down_blocks), _ptr(down_scales), _ptr(down_bias), int(T),
+                                   ctypes.c_void_p(out_host.data_ptr()), _stream(stream)), "moe_forward_hostio")
+
+
+def moe_debug_dequant(blocks, scales, rows: int, cols: int, out, stream=None) -> None:
+    _check(_lib.moe_debug_dequant(_ptr(blocks), _ptr(scales), int(rows), int(cols), _ptr(out), _stream(stream)),
+           "moe_debug_dequant")
+
+
+def moe_debug_decode_codes(codes, n: int, out, stream=None) -> None:
+    _check(_lib.moe_debug_decode_codes(_ptr(codes), int(n), _ptr(out), _stream(stream)), "moe_debug_decode_codes")
+
+
+def moe_debug_route(h, x, router_w, router_b, T: int, idx=None, w=None, perm=None, offsets=None,
+                    stream=None) -> None:
+    _check(_lib.moe_debug_route(h, _ptr(x), _ptr(router_w), _ptr(router_b), int(T), _ptr(idx), _ptr(w), _ptr(perm),
+                                _ptr(offsets), _stream(stream)), "moe_debug_route")
+
+
+class MoeLayer:
+    """Owns a handle and a set of device weights; ``forward(x)`` returns a bf16 [T, H] tensor."""
+
+    ORDER = ("router_w", "router_b", "gate_up_blocks", "gate_up_scales", "gate_up_bias", "down_blocks",
+             "down_scales", "down_bias")
+
+    def __init__(self, H: int, I: int, E: int, top_k: int, max_T: int, weights: dict):
+        self.H, self.I, self.E, self.k, self.max_T = H, I, E, top_k, max_T
+        self.h = moe_create(H, I, E, top_k, max_T)
+        self.weights = [weights[n] for n in self.ORDER]
+
+    def set_option(self, opt: int, value: int) -> None:
+        moe_set_option(self.h, opt, value)
+
+    def forward(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x.device)
+        moe_forward(self.h, x, *self.weights, T, out, stream)
+        return out
+
+    def close(self) -> None:
+        if self.h is not None:
+            moe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,88 @@
+"""The C-ABI library on the CPU machine: it loads, exports every declared symbol, and validates arguments
+before touching the GPU (no compute calls are made here)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mxfp4_expert_ffn_bias_b200 import build
+    build.build()
+    from mxfp4_expert_ffn_bias_b200 import moe
+    return moe
+
+
+def test_header_declares_the_abi():
+    names = _declared()
+    for n in ("moe_create", "moe_forward", "moe_destroy", "moe_status_string", "moe_set_option",
+              "moe_debug_dequant", "moe_debug_route", "moe_sync_status", "moe_forward_hostio", "moe_stage_times",
+              "moe_debug_decode_codes"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(\S+)", out))
+    for n in _declared():
+        assert n in exported, n
+        assert hasattr(lib._lib, n)
+    # nothing but the ABI is exported from our own code
+    ours = {s for s in exported if s.startswith("moe_")}
+    assert ours == set(_declared())
+    # the binding wraps every declared symbol
+    assert set(lib.SIGNATURES) == set(_declared())
+
+
+def test_status_strings(lib):
+    assert lib.moe_status_string(0) == "MOE_OK"
+    assert lib.moe_status_string(5) == "MOE_ERR_DEVICE_TIMEOUT"
+    assert lib.moe_status_string(99) == "MOE_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("args", [
+    (2880, 2880, 32, 4, 0),      # max_T < 1
+    (2880, 2880, 32, 0, 8),      # top_k < 1
+    (2880, 2880, 32, 9, 8),      # top_k > 8
+    (2880, 2880, 3, 4, 8),       # E < top_k
+    (2880, 2880, 257, 4, 8),     # E > 256
+    (2880 + 32, 2880, 32, 4, 8),  # H % 64
+    (2880, 100, 32, 4, 8),       # I % 64
+])
+def test_create_rejects_bad_shapes_before_cuda(lib, args):
+    h = ctypes.c_void_p()
+    assert lib._lib.moe_create(*args, ctypes.byref(h)) == lib.MOE_ERR_INVALID_ARG
+    assert h.value is None
+
+
+def test_null_handle_and_pointer_checks(lib):
+    P = ctypes.c_void_p
+    assert lib._lib.moe_forward(None, *([P(16)] * 9), 1, P(16), None) == lib.MOE_ERR_INVALID_ARG
+    assert lib._lib.moe_set_option(None, 1, 0) == lib.MOE_ERR_INVALID_ARG
+    assert lib._lib.moe_sync_status(None) == lib.MOE_ERR_INVALID_ARG
+    assert lib._lib.moe_debug_dequant(None, None, 1, 32, None, None) == lib.MOE_ERR_INVALID_ARG
+    assert lib._lib.moe_debug_dequant(P(16), P(16), 1, 48, P(16), None) == lib.MOE_ERR_INVALID_ARG  # cols % 32
+    assert lib._lib.moe_debug_dequant(P(8), P(16), 1, 32, P(16), None) == lib.MOE_ERR_INVALID_ARG  # misaligned
+    assert lib._lib.moe_destroy(None) == lib.MOE_OK
+    assert lib._lib.moe_stage_times(None, None, 4, None) == lib.MOE_ERR_INVALID_ARG
+
+
+def test_create_without_gpu_reports_cuda_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    h = ctypes.c_void_p()
+    assert lib._lib.moe_create(256, 256, 8, 2, 16, ctypes.byref(h)) == lib.MOE_ERR_CUDA

@@ -1,0 +1,288 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle.
+
+Bars (written here, per quantity):
+  * dequantised weights and selected expert indices: bit-exact;
+  * the routing permutation (a stable counting sort) and offsets: exact;
+  * routing weights: |w_gpu - w_ref| <= 1e-5 (fp32 softmax of fp32 logits);
+  * layer outputs: max|gpu - ref| <= 2e-2 * max|ref| + 1e-3 and
+    sum|gpu - ref| / sum|ref| <= 5e-3.
+"""
+
+import os
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gen.synth import CONFIGS, Config, make_inputs
+from tests.gpu_util import assert_parity, bf16_dev_to_f64, run_forward, score, to_device
+
+pytestmark = pytest.mark.gpu
+
+NCPU = os.cpu_count() or 1
+
+
+@pytest.fixture(scope="module")
+def moe():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from mxfp4_expert_ffn_bias_b200 import build
+    build.build()
+    from mxfp4_expert_ffn_bias_b200 import moe as m
+    torch.cuda.set_device(0)
+    return m
+
+
+_cache = {}
+
+
+def inputs_for(name_or_cfg, seed=0, T=None):
+    key = (getattr(name_or_cfg, "name", name_or_cfg), seed, T)
+    if key not in _cache:
+        if len(_cache) > 2:
+            _cache.clear()
+        _cache[key] = make_inputs(name_or_cfg, seed=seed, T=T, margin_fn=oracle.router_margins)
+    return _cache[key]
+
+
+def cfg_of(name_or_cfg):
+    return CONFIGS[name_or_cfg] if isinstance(name_or_cfg, str) else name_or_cfg
+
+
+# ---------------------------------------------------------------- dequant and FP4 conversion
+
+
+def test_debug_dequant_exhaustive_bit_exact(moe):
+    scales_range = np.arange(2, 253, dtype=np.uint8)
+    nb = 16
+    blocks = np.ascontiguousarray(
+        np.broadcast_to(np.arange(256, dtype=np.uint8).reshape(1, nb, 16), (scales_range.size, nb, 16)))
+    scales = np.ascontiguousarray(np.broadcast_to(scales_range[:, None], (scales_range.size, nb)))
+    ref, bad = oracle.dequant_bf16(blocks, scales)
+    assert bad == 0
+    out = torch.empty((scales_range.size, nb * 32), dtype=torch.int16, device="cuda")
+    moe.moe_debug_dequant(torch.from_numpy(blocks).cuda(), torch.from_numpy(scales).cuda(), scales_range.size,
+                          nb * 32, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+
+
+def test_debug_dequant_random_gpt_oss_rows_bit_exact(moe):
+    rng = np.random.default_rng(1)
+    R, C = 777, 2880
+    blocks = rng.integers(0, 256, (R, C // 32, 16), dtype=np.uint8)
+    scales = rng.integers(2, 253, (R, C // 32), dtype=np.uint8)
+    ref, bad = oracle.dequant_bf16(blocks, scales)
+    assert bad == 0
+    out = torch.empty((R, C), dtype=torch.int16, device="cuda")
+    moe.moe_debug_dequant(torch.from_numpy(blocks).cuda(), torch.from_numpy(scales).cuda(), R, C, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), ref)
+
+
+def test_decode_fp4_converter_exact(moe):
+    codes = torch.arange(256, dtype=torch.uint8, device="cuda")  # 64 words: the decode kernels read words
+    out = torch.empty(256, dtype=torch.int32, device="cuda")
+    moe.moe_debug_decode_codes(codes, 256, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().view(np.uint32)
+    lo = (got & 0xFFFF).astype(np.uint16).view(np.float16).astype(np.float64)
+    hi = (got >> 16).astype(np.uint16).view(np.float16).astype(np.float64)
+    for b in range(256):
+        assert lo[b] == oracle.e2m1_value(b & 15) and np.signbit(lo[b]) == np.signbit(oracle.e2m1_value(b & 15))
+        assert hi[b] == oracle.e2m1_value(b >> 4) and np.signbit(hi[b]) == np.signbit(oracle.e2m1_value(b >> 4))
+
+
+# ---------------------------------------------------------------- routing
+
+
+@pytest.mark.parametrize("name", ["tiny", "gpt-oss-20b-decode", "gpt-oss-120b-decode", "gpt-oss-20b-prefill",
+                                  "gpt-oss-120b-prefill-zipf"])
+def test_route_topk_softmax_and_permutation(moe, name):
+    cfg = cfg_of(name)
+    inp = inputs_for(name)
+    T = inp["x"].shape[0]
+    dev = to_device(inp)
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
+    try:
+        idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+        perm = torch.empty(T * cfg.k, dtype=torch.int32, device="cuda")
+        offs = torch.empty(cfg.E + 1, dtype=torch.int32, device="cuda")
+        moe.moe_debug_route(h, dev["x"], dev["router_w"], dev["router_b"], T, idx, w, perm, offs)
+        torch.cuda.synchronize()
+    finally:
+        moe.moe_destroy(h)
+    lg = oracle.router_logits(inp["x"], inp["router_w"], inp["router_b"])
+    ref_idx, ref_w = oracle.topk_softmax(lg, cfg.k)
+    got_idx = idx.cpu().numpy()
+    assert np.array_equal(got_idx, ref_idx)
+    assert np.abs(w.cpu().numpy() - ref_w).max() <= 1e-5
+    flat = ref_idx.ravel()
+    assert np.array_equal(perm.cpu().numpy(), np.argsort(flat, kind="stable"))
+    counts = np.bincount(flat, minlength=cfg.E)
+    assert np.array_equal(offs.cpu().numpy(), np.concatenate([[0], np.cumsum(counts)]))
+
+
+# ---------------------------------------------------------------- whole layer
+
+
+def _run_layer(moe, name_or_cfg, path, T=None, seed=0, tokens=None, repeat=1, variant=None):
+    cfg = cfg_of(name_or_cfg)
+    inp = inputs_for(name_or_cfg, seed=seed, T=T)
+    T = inp["x"].shape[0]
+    dev = to_device(inp)
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
+    outs = []
+    try:
+        moe.moe_set_option(h, moe.MOE_OPT_PATH, path)
+        if variant is not None:
+            moe.moe_set_option(h, moe.MOE_OPT_DECODE_KERNEL, variant)
+        for _ in range(repeat):
+            outs.append(run_forward(moe, h, dev, T, cfg.H))
+        torch.cuda.synchronize()
+        assert moe.moe_sync_status(h) == moe.MOE_OK
+    finally:
+        moe.moe_destroy(h)
+    got = [bf16_dev_to_f64(o) for o in outs]
+    ref, _, _ = oracle.moe_forward(inp, cfg.k, tokens=tokens, threads=NCPU)
+    sel = got[0] if tokens is None else got[0][np.asarray(tokens)]
+    return sel, ref, got
+
+
+# (path, decode engine): 1 = routed-expert GEMV (engine 0 CUDA-core FMA, 1 warp MMA), 2 = grouped tcgen05 GEMM
+PATHS = [(1, 0), (1, 1), (2, None)]
+
+
+@pytest.mark.parametrize("path,variant", PATHS)
+def test_tiny_layer_all_paths(moe, path, variant):
+    got, ref, _ = _run_layer(moe, "tiny", path, variant=variant)
+    assert_parity(got, ref, f"tiny path={path} variant={variant}")
+
+
+@pytest.mark.parametrize("path,variant", PATHS)
+def test_tiny_shapes_many_tiles_ragged(moe, path, variant):
+    """T=1000 on the tiny layer: ~250 rows per expert -> several M tiles and a ragged last tile;
+    also exercises the large-T routing (chunked stable scatter) and multi-pass GEMVs."""
+    cfg = Config("tiny-T1000", T=1000, H=256, I=256, E=8, k=2, scale_lo=119, scale_hi=123, router_bias="normal")
+    got, ref, _ = _run_layer(moe, cfg, path, variant=variant)
+    assert_parity(got, ref, f"tiny-T1000 path={path}")
+
+
+@pytest.mark.parametrize("T", [1, 3, 64, 65])
+@pytest.mark.parametrize("path,variant", PATHS)
+def test_token_counts_around_routing_switch(moe, T, path, variant):
+    """T <= 64 routes in one launch, T > 64 through the chunked scatter; both must agree with the oracle."""
+    got, ref, _ = _run_layer(moe, "tiny", path, T=T, variant=variant)
+    assert_parity(got, ref, f"T={T} path={path}")
+
+
+@pytest.mark.parametrize("path,variant", PATHS)
+def test_all_experts_selected_and_single_expert(moe, path, variant):
+    for E, k in ((4, 4), (6, 1)):
+        cfg = Config(f"e{E}k{k}", T=40, H=128, I=192, E=E, k=k, scale_lo=118, scale_hi=124, router_bias="normal")
+        got, ref, _ = _run_layer(moe, cfg, path, variant=variant)
+        assert_parity(got, ref, f"E={E} k={k} path={path}")
+
+
+@pytest.mark.parametrize("path,variant", PATHS)
+def test_gpt_oss_20b_decode(moe, path, variant):
+    got, ref, _ = _run_layer(moe, "gpt-oss-20b-decode", path, variant=variant)
+    assert_parity(got, ref, f"20b decode path={path} variant={variant}")
+
+
+@pytest.mark.parametrize("path,variant", PATHS)
+def test_gpt_oss_120b_decode_sampled(moe, path, variant):
+    tokens = [0, 1, 2, 17, 31, 40, 55, 62, 63]
+    got, ref, _ = _run_layer(moe, "gpt-oss-120b-decode", path, tokens=tokens, variant=variant)
+    assert_parity(got, ref, f"120b decode path={path} variant={variant}")
+
+
+def _sample(T, n=16, seed=0):
+    rng = np.random.default_rng(seed)
+    return sorted(set([0, 1, T - 1] + rng.choice(T, n, replace=False).tolist()))
+
+
+def test_gpt_oss_20b_prefill_sampled_and_deterministic(moe):
+    T = CONFIGS["gpt-oss-20b-prefill"].T
+    tokens = _sample(T)
+    got, ref, outs = _run_layer(moe, "gpt-oss-20b-prefill", 0, tokens=tokens, repeat=2)
+    assert_parity(got, ref, "20b prefill")
+    assert np.array_equal(outs[0], outs[1])  # same inputs, same bits
+
+
+def test_gpt_oss_120b_prefill_zipf_sampled(moe):
+    T = CONFIGS["gpt-oss-120b-prefill-zipf"].T
+    inp = inputs_for("gpt-oss-120b-prefill-zipf")
+    lg = oracle.router_logits(inp["x"][:2048], inp["router_w"], inp["router_b"])
+    idx, _ = oracle.topk_softmax(lg, 4)
+    hot = int(np.argmax(np.bincount(idx.ravel(), minlength=128)))
+    hot_tok = int(np.nonzero((idx == hot).any(1))[0][0])
+    tokens = sorted(set(_sample(T, 14, seed=3) + [hot_tok]))
+    got, ref, _ = _run_layer(moe, "gpt-oss-120b-prefill-zipf", 0, tokens=tokens)
+    assert_parity(got, ref, "120b prefill zipf")
+
+
+def test_decode_and_prefill_paths_agree(moe):
+    """Routed-only (decode GEMV) and grouped-GEMM evaluation of the same layer both meet the bar and agree."""
+    a, ref, _ = _run_layer(moe, "gpt-oss-20b-decode", 1)
+    b, _, _ = _run_layer(moe, "gpt-oss-20b-decode", 2)
+    c, _, _ = _run_layer(moe, "gpt-oss-20b-decode", 1, variant=0)
+    assert_parity(c, ref, "decode cuda-core engine")
+    assert_parity(a, ref, "decode")
+    assert_parity(b, ref, "prefill")
+    s = score(a, b)
+    assert s["max_err"] <= 2e-2 * s["max_ref"] + 1e-3
+
+
+def test_hostio_matches_device_path(moe):
+    cfg = CONFIGS["tiny"]
+    inp = inputs_for("tiny")
+    dev = to_device(inp)
+    T = cfg.T
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
+    try:
+        out_dev = run_forward(moe, h, dev, T, cfg.H)
+        torch.cuda.synchronize()
+        x_host = torch.from_numpy(inp["x"].view(np.int16).copy()).pin_memory()
+        out_host = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
+        moe.moe_forward_hostio(h, x_host, dev["router_w"], dev["router_b"], dev["gate_up_blocks"],
+                               dev["gate_up_scales"], dev["gate_up_bias"], dev["down_blocks"], dev["down_scales"],
+                               dev["down_bias"], T, out_host)
+    finally:
+        moe.moe_destroy(h)
+    assert np.array_equal(out_host.numpy(), out_dev.view(torch.int16).cpu().numpy())
+
+
+def test_invalid_token_counts_rejected(moe):
+    cfg = CONFIGS["tiny"]
+    dev = to_device(inputs_for("tiny"))
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, 16)
+    try:
+        for T in (0, 17):
+            with pytest.raises(moe.MoeError) as ei:
+                moe.moe_forward(h, dev["x"], dev["router_w"], dev["router_b"], dev["gate_up_blocks"],
+                                dev["gate_up_scales"], dev["gate_up_bias"], dev["down_blocks"], dev["down_scales"],
+                                dev["down_bias"], T, torch.empty((16, cfg.H), dtype=torch.bfloat16, device="cuda"))
+            assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    finally:
+        moe.moe_destroy(h)
+
+
+def test_stage_times_reported(moe):
+    cfg = CONFIGS["tiny"]
+    dev = to_device(inputs_for("tiny"))
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, cfg.T)
+    try:
+        moe.moe_set_option(h, moe.MOE_OPT_STAGE_EVENTS, 4)
+        for _ in range(3):
+            run_forward(moe, h, dev, cfg.T, cfg.H)
+        ms, n = moe.moe_stage_times(h)
+        ms2, n2 = moe.moe_stage_times(h)
+    finally:
+        moe.moe_destroy(h)
+    assert n == 3 and len(ms) == 4 and all(m >= 0 for m in ms) and sum(ms) > 0
+    assert n2 == 0 and sum(ms2) == 0
