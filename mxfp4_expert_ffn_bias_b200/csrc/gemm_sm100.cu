@@ -1,32 +1,41 @@
 // Prefill path: grouped MXFP4 GEMMs on the 5th-generation tensor cores.
 //
-// D[rows of expert e, n] = A[rows, K] . dequant(W[e])[n, K]^T, for every
-// expert with routed rows, in one persistent launch. A is the bf16 token
-// matrix in permuted (expert-grouped) order: the gathered x for gate_up and
-// the SwiGLU output for down. W is an MXFP4 tensor (E2M1 codes two per byte,
-// one E8M0 scale per 32 K elements; ZeroModels GPT-OSS docs, "MXFP4 experts").
+// For every expert e with routed rows, and every tile of its output features,
+//   D[n, t] = dequant(W[e])[n, :] . A[t, :]        (n: output feature, t: routed token row)
+// in one persistent launch. W is an MXFP4 tensor (E2M1 codes two per byte,
+// one E8M0 scale per 32 K elements; ZeroModels GPT-OSS docs, "MXFP4 experts");
+// A is the bf16 token matrix in expert-grouped (permuted) order: the gathered
+// x for gate_up, the SwiGLU output for down.
+//
+// The weights are the MMA's M operand and live in TENSOR MEMORY: dequant warps
+// convert each 128-row x 64-column packed tile exactly to bf16 in registers
+// (mx_dequant8_bf16) and write it with tcgen05.st into a ring of TMEM stages;
+// tcgen05.mma (kind::f16, A from TMEM, B = 192 token rows from shared memory)
+// accumulates D[128 x 192] in fp32 in TMEM. The dequantised tile never touches
+// shared memory, and each converted weight element serves 192 token rows.
 //
 // Per CTA (one per SM), warp-specialised:
-//   warp 4      TMA producer: A tile (128 x 64 bf16, 128B swizzle) and the
-//               packed weight tile (BN x 32 bytes) per K step into a ring of
-//               STAGES stages; the tile's E8M0 scales (BN x K/32 bytes,
-//               contiguous in memory) with one bulk copy per output tile.
-//   warps 6-9   dequantise the packed tile exactly to bf16 (mx_dequant8_bf16)
-//               into the stage's B tile, in the same 128B-swizzled K-major
-//               layout TMA gives A.
-//   warp 5      one thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32,
-//               M=128, N=BN, K=16) into a TMEM accumulator; commits free the
-//               stage and, at the end of a tile, hand the accumulator over.
-//   warps 0-3   epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
-//               32w..32w+31 = tile rows), add the bias and either
-//                 gate_up: de-interleave (even columns = gate, odd = up; MaxText
-//                 PR 2647 "1 Support many-to-one transform"), apply the clamped
-//                 SwiGLU and store bf16 act[row, n/2], or
-//                 down: scale by the routing weight and store fp32 rows of the
-//                 slot buffer at the row's (token, slot) pair index.
-// Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile overlap
-// the main loop of the next. Every wait is bounded; a wait that gives up sets
-// the status word and the CTA winds down.
+//   warp 4      TMA producer: token tile (192 x 64 bf16, 128B swizzle) and the
+//               packed weight tile (128 x 32 bytes) per K step into a ring of
+//               4 shared-memory stages; the tile's E8M0 scales (128 x K/32
+//               bytes, contiguous) with one bulk copy per output tile.
+//   warps 6..   dequant (8 warps): warp w converts part (w-6)/4 of each K step
+//               for TMEM sub-partition w % 4 (lanes = weight rows); converting
+//               step k+1 overlaps the TMEM store of step k.
+//   warp 5      one thread issues 4 MMAs (K = 16 each) per stage, commits to
+//               free the stage and, after the last K step, hands the
+//               accumulator to the epilogue.
+//   warps 0-3   epilogue: tcgen05.ld (lane = weight row, column = token), add
+//               the bias and either
+//                 gate_up: pair gate row 2i with up row 2i+1 (adjacent lanes;
+//                 MaxText PR 2647 "1 Support many-to-one transform"), apply the
+//                 clamped SwiGLU and store bf16 act[t, i], or
+//                 down: scale by the token's routing weight and store the fp32
+//                 slot row of the token's (token, slot) pair.
+// Two TMEM accumulators (2 x 192 columns) plus 4 TMEM A stages (4 x 32
+// columns) use all 512 columns, so the epilogue of one tile overlaps the main
+// loop of the next. Every wait is bounded; a wait that gives up sets the
+// status word and the CTA winds down.
 #include <cstdio>
 
 #include "common.cuh"
@@ -37,30 +46,47 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 0, kProdWarp = 4, kMmaWarp = 5, kDeqWarp0 = 6;
+constexpr int kWM = 128;                    // weight rows per tile (MMA M, TMEM lanes)
+constexpr int kTN = kBM;                    // token rows per tile (MMA N)
+constexpr int kStages = 4;
+#ifndef MOE_DEQ_WARPS
+#define MOE_DEQ_WARPS 8  // measured: 8 (900 us) beat 16 (972 us) on the 20b prefill gate_up
+#endif
+constexpr int kDeqWarps = MOE_DEQ_WARPS;    // 8 or 16: 2 or 4 per TMEM sub-partition
+constexpr int kDeqSplit = kDeqWarps / 4;    // warps sharing one sub-partition split each K step
+constexpr int kDeqCols = kBK / 2 / kDeqSplit;  // TMEM columns (bf16 pairs) per dequant thread per step
+static_assert(kDeqSplit == 2 || kDeqSplit == 4, "dequant split");
+constexpr int kProdWarp = 4, kMmaWarp = 5, kDeqWarp0 = 6;  // warps 0-3: epilogue
+constexpr int kThreads = 32 * (kDeqWarp0 + kDeqWarps);
+constexpr int kAccCols = kTN;               // fp32 columns of one accumulator
+constexpr int kAStageCols = kBK / 2;        // TMEM columns of one bf16 A stage (64 K values)
+constexpr int kAColBase = 2 * kAccCols;     // A stages follow the two accumulators
+constexpr int kTmemCols = 512;
+static_assert(kAColBase + kStages * kAStageCols <= kTmemCols, "TMEM budget");
 constexpr int kMaxE = 256;
 
-template <int BN, int STAGES>
-struct Smem {
-  static constexpr int kA = kBM * 128;  // bytes of one A stage
-  static constexpr int kB = BN * 128;   // bytes of one dequantised B stage
-  static constexpr int kP = BN * 32;    // bytes of one packed stage
-  static constexpr int offA = 0;
-  static constexpr int offB = offA + STAGES * kA;
-  static constexpr int offP = offB + STAGES * kB;
-  static constexpr int offSC = offP + STAGES * kP;  // 2 scale buffers of BN*KB bytes (runtime size)
+constexpr int kTokBytes = kTN * 128;        // one token stage (64 bf16 per row)
+constexpr int kPackBytes = kWM * 32;        // one packed weight stage (32 bytes per row)
+constexpr int kOffTok = 0;
+constexpr int kOffPack = kOffTok + kStages * kTokBytes;
+constexpr int kOffEpi = kOffPack + kStages * kPackBytes;  // epilogue staging (see Epi)
+struct Epi {
+  uint16_t act[4][16][16];  // per epilogue warp: 16 tokens x 16 SwiGLU outputs (bf16), transposed for stores
+  int pair[2][kBM];         // per accumulator buffer: (token, slot) pair of each token row of the tile
+  float w[2][kBM];          // its routing weight
 };
+constexpr int kOffSc = kOffEpi + (int)((sizeof(Epi) + 127) / 128 * 128);  // 2 scale buffers of kWM * KB bytes
 
 struct __align__(8) Bars {
-  uint64_t full_ab[8];
-  uint64_t full_b[8];
-  uint64_t empty[8];
+  uint64_t full_ab[kStages];   // TMA landed (token + packed tiles)
+  uint64_t full_b[kStages];    // TMEM A stage written by the dequant warps
+  uint64_t empty[kStages];     // MMAs of the stage done
   uint64_t sc_full[2];
   uint64_t sc_empty[2];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
+  uint64_t epi_sync[2];        // the 4 epilogue warps staged the tile's token metadata
   uint32_t tmem_base;
   int abort_flag;
   int counts[kMaxE];
@@ -68,13 +94,7 @@ struct __align__(8) Bars {
   int mt_off[kMaxE + 1];
 };
 
-// Dynamic shared memory of one CTA. At least 116 KB, so that no two CTAs of
-// this kernel share an SM (each allocates all 512 TMEM columns).
-template <int BN, int STAGES>
-size_t smem_total(int K) {
-  const size_t need = 1024 + Smem<BN, STAGES>::offSC + 2 * (size_t)BN * (K / 32) + sizeof(Bars) + 64;
-  return need < 116 * 1024 ? 116 * 1024 : need;
-}
+size_t smem_total(int K) { return 1024 + kOffSc + 2 * (size_t)kWM * (K / 32) + sizeof(Bars) + 64; }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -84,9 +104,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Bounded, abortable wait used by every role: gives up after `limit_us`
 // microseconds of wall time (or as soon as another role gave up), raising the
-// status word and the CTA's abort flag.
-// With abortable = false (used to drain copies and MMAs still in flight before
-// the CTA exits) only the time limit ends the wait.
+// status word and the CTA's abort flag. With abortable = false (used to drain
+// copies and MMAs still in flight before the CTA exits) only the time limit
+// ends the wait.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, long long limit_us, volatile int* abort_flag,
                                          unsigned* status, bool abortable = true) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -108,6 +128,9 @@ struct TileInfo {
   int e, lm, nt, row0, valid;
 };
 
+// Tile t -> (expert, token tile lm, weight tile nt). Tiles are ordered token-
+// tile-major so that the CTAs working at the same time share one expert's
+// weights (L2 reuse) and one token tile per group of weight tiles.
 __device__ __forceinline__ TileInfo decode_tile(const Bars& b, int E, int NT, int t) {
   TileInfo ti;
   const int mt = t / NT;
@@ -119,29 +142,28 @@ __device__ __forceinline__ TileInfo decode_tile(const Bars& b, int E, int NT, in
   }
   ti.e = lo;
   ti.lm = mt - b.mt_off[lo];
-  ti.row0 = b.offsets[lo] + ti.lm * kBM;
-  ti.valid = min(kBM, b.counts[lo] - ti.lm * kBM);
+  ti.row0 = b.offsets[lo] + ti.lm * kTN;
+  ti.valid = min(kTN, b.counts[lo] - ti.lm * kTN);
   return ti;
 }
 
 __device__ __forceinline__ float silu_clamped(float hg, float hu) {
   const float g = fminf(hg, 7.f);
   const float u = fminf(fmaxf(hu, -7.f), 7.f);
-  return (u + 1.f) * g * (1.f / (1.f + expf(-1.702f * g)));
+  return (u + 1.f) * g * (1.f / (1.f + __expf(-1.702f * g)));
 }
 
-template <int BN, int STAGES, bool kGateUp>
+template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_mxfp4_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapP,
                        GemmArgs a) {
-  using L = Smem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int KB = a.K / 32;
   const int KT = a.K / kBK;
-  const int NT = a.N / BN;
-  const int scbytes = BN * KB;
-  Bars& b = *reinterpret_cast<Bars*>(smem + L::offSC + 2 * scbytes);
+  const int NT = (a.N + kWM - 1) / kWM;
+  const int scbytes = kWM * KB;
+  Bars& b = *reinterpret_cast<Bars*>(smem + kOffSc + 2 * scbytes);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_flag = &b.abort_flag;
 
@@ -151,23 +173,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     b.mt_off[i] = a.mt_off[i];
   }
   if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&b.full_ab[s], 1);
-      mbar_init(&b.full_b[s], 4);
+      mbar_init(&b.full_b[s], kDeqWarps);
       mbar_init(&b.empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b.sc_full[i], 1);
-      mbar_init(&b.sc_empty[i], 4);
+      mbar_init(&b.sc_empty[i], kDeqWarps);
       mbar_init(&b.acc_full[i], 1);
       mbar_init(&b.acc_empty[i], 4);
     }
     mbar_init(&b.drain, 1);
+    mbar_init(&b.epi_sync[0], 4);
+    mbar_init(&b.epi_sync[1], 4);
     b.abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&b.tmem_base, 512);
+    tmem_alloc(&b.tmem_base, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -183,53 +207,86 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tc) {
         const TileInfo ti = decode_tile(b, a.E, NT, t);
+        const int n0 = ti.nt * kWM;
+        const int wrows = min(kWM, a.N - n0);
         const int sb = tc & 1;
         if (tc >= 2) ok = wait_bar(&b.sc_empty[sb], ((tc >> 1) - 1) & 1, lim, abort_flag, a.status);
         if (!ok) break;
-        uint8_t* scdst = smem + L::offSC + sb * scbytes;
-        mbar_arrive_expect_tx(&b.sc_full[sb], scbytes);
-        bulk_load(scdst, a.scales + ((size_t)ti.e * a.N + (size_t)ti.nt * BN) * KB, scbytes, &b.sc_full[sb]);
-        const int prow = ti.e * a.N + ti.nt * BN;
+        mbar_arrive_expect_tx(&b.sc_full[sb], wrows * KB);
+        bulk_load(smem + kOffSc + sb * scbytes, a.scales + ((size_t)ti.e * a.N + n0) * KB, wrows * KB,
+                  &b.sc_full[sb]);
+        const int prow = ti.e * a.N + n0;
         for (int kt = 0; kt < KT; ++kt, ++it) {
-          const int s = it % STAGES;
-          ok = wait_bar(&b.empty[s], ((it / STAGES) & 1) ^ 1, lim, abort_flag, a.status);
+          const int s = it % kStages;
+          ok = wait_bar(&b.empty[s], ((it / kStages) & 1) ^ 1, lim, abort_flag, a.status);
           if (!ok) break;
-          mbar_arrive_expect_tx(&b.full_ab[s], L::kA + L::kP);
-          tma_load_2d(smem + L::offA + s * L::kA, &mapA, &b.full_ab[s], kt * kBK, ti.row0);
-          tma_load_2d(smem + L::offP + s * L::kP, &mapP, &b.full_ab[s], kt * (kBK / 2), prow);
+          mbar_arrive_expect_tx(&b.full_ab[s], kTokBytes + kPackBytes);
+          tma_load_2d(smem + kOffTok + s * kTokBytes, &mapA, &b.full_ab[s], kt * kBK, ti.row0);
+          tma_load_2d(smem + kOffPack + s * kPackBytes, &mapP, &b.full_ab[s], kt * (kBK / 2), prow);
         }
       }
       // Drain: wait (bounded) for copies still in flight before the CTA may exit.
-      for (int j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-        wait_bar(&b.full_ab[j % STAGES], (j / STAGES) & 1, lim, abort_flag, a.status, false);
+      for (int j = (it > kStages ? it - kStages : 0); j < it; ++j)
+        wait_bar(&b.full_ab[j % kStages], (j / kStages) & 1, lim, abort_flag, a.status, false);
       for (int j = (tc > 2 ? tc - 2 : 0); j < tc; ++j)
         wait_bar(&b.sc_full[j & 1], (j >> 1) & 1, lim, abort_flag, a.status, false);
     }
   } else if (warp >= kDeqWarp0) {
-    const int dt = tid - kDeqWarp0 * 32;  // 0..127
+    // Thread: weight row r = 32 (warp % 4) + lane of the tile (its TMEM lane),
+    // part h = (warp - 6) / 4 of each 64-wide K step: kDeqCols TMEM columns
+    // (2 kDeqCols bf16) from kDeqCols packed bytes. The loop is software-
+    // pipelined: step k+1 is loaded and converted while step k's TMEM store
+    // drains.
+    const int sub = warp & 3, h = (warp - kDeqWarp0) >> 2;
+    const int r = sub * 32 + lane;
+    const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16) + kAColBase + h * kDeqCols;
+    const int pk_off = r * 32 + h * kDeqCols;        // byte offset of this thread's packed bytes
+    const int sc_blk = (h * kDeqCols) / 16;          // MX block of the step (0 or 1)
     int it = 0, tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tc) {
       const int sb = tc & 1;
       ok = wait_bar(&b.sc_full[sb], (tc >> 1) & 1, lim, abort_flag, a.status);
       if (!ok) break;
-      const uint8_t* sc = smem + L::offSC + sb * scbytes;
-      for (int kt = 0; kt < KT; ++kt, ++it) {
-        const int s = it % STAGES;
-        ok = wait_bar(&b.full_ab[s], (it / STAGES) & 1, lim, abort_flag, a.status);
-        if (!ok) break;
-        const uint8_t* P = smem + L::offP + s * L::kP;
-        uint8_t* B = smem + L::offB + s * L::kB;
-#pragma unroll 4
-        for (int c = dt; c < BN * 8; c += 128) {
-          const int r = c >> 3, q = c & 7;
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(P + r * 32 + q * 4);
-          const uint32_t sv = sc[r * KB + kt * 2 + (q >> 2)];
-          *reinterpret_cast<uint4*>(B + r * 128 + ((q ^ (r & 7)) << 4)) = mx_dequant8_bf16(w, sv);
+      const uint8_t* sc = smem + kOffSc + sb * scbytes + r * KB + sc_blk;
+      uint32_t va[kDeqCols], vb[kDeqCols];  // step k in va (being stored), step k+1 converted into vb
+      auto convert = [&](int kt, int s, uint32_t* v) {
+        const uint32_t sv = sc[kt * 2];
+        const uint8_t* src = smem + kOffPack + s * kPackBytes + pk_off;
+        if constexpr (kDeqCols == 16) {
+          const uint4 pk = *reinterpret_cast<const uint4*>(src);
+          const uint4 q0 = mx_dequant8_bf16(pk.x, sv), q1 = mx_dequant8_bf16(pk.y, sv);
+          const uint4 q2 = mx_dequant8_bf16(pk.z, sv), q3 = mx_dequant8_bf16(pk.w, sv);
+          v[0] = q0.x, v[1] = q0.y, v[2] = q0.z, v[3] = q0.w, v[4] = q1.x, v[5] = q1.y, v[6] = q1.z, v[7] = q1.w;
+          v[8] = q2.x, v[9] = q2.y, v[10] = q2.z, v[11] = q2.w, v[12] = q3.x, v[13] = q3.y, v[14] = q3.z,
+          v[15] = q3.w;
+        } else {
+          const uint2 pk = *reinterpret_cast<const uint2*>(src);
+          const uint4 q0 = mx_dequant8_bf16(pk.x, sv), q1 = mx_dequant8_bf16(pk.y, sv);
+          v[0] = q0.x, v[1] = q0.y, v[2] = q0.z, v[3] = q0.w, v[4] = q1.x, v[5] = q1.y, v[6] = q1.z, v[7] = q1.w;
         }
-        fence_proxy_async_smem();
+      };
+      ok = wait_bar(&b.full_ab[it % kStages], (it / kStages) & 1, lim, abort_flag, a.status);
+      if (!ok) break;
+      convert(0, it % kStages, va);
+      for (int kt = 0; kt < KT; ++kt, ++it) {
+        const int s = it % kStages;
+        if constexpr (kDeqCols == 16) tmem_st16(t_lane + s * kAStageCols, va);
+        else tmem_st8(t_lane + s * kAStageCols, va);
+        const bool more = kt + 1 < KT;
+        if (more) {  // convert the next step while this store drains
+          ok = wait_bar(&b.full_ab[(it + 1) % kStages], ((it + 1) / kStages) & 1, lim, abort_flag, a.status);
+          if (ok) convert(kt + 1, (it + 1) % kStages, vb);
+        }
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.full_b[s]);
+        if (!ok) break;
+        if (more) {
+#pragma unroll
+          for (int i = 0; i < kDeqCols; ++i) va[i] = vb[i];
+        }
       }
       if (!ok) break;
       __syncwarp();
@@ -237,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(kBM, BN);
+      constexpr uint32_t idesc = idesc_bf16(kWM, kTN);
       int it = 0, tc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tc) {
@@ -245,20 +302,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_bar(&b.acc_empty[ab], ((tc >> 1) & 1) ^ 1, lim, abort_flag, a.status);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * 256;
+        const uint32_t d_tmem = tmem_base + ab * kAccCols;
         for (int kt = 0; kt < KT; ++kt, ++it) {
-          const int s = it % STAGES;
-          const uint32_t par = (it / STAGES) & 1;
+          const int s = it % kStages;
+          const uint32_t par = (it / kStages) & 1;
           ok = wait_bar(&b.full_ab[s], par, lim, abort_flag, a.status) &&
                wait_bar(&b.full_b[s], par, lim, abort_flag, a.status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + L::offA + s * L::kA);
-          const uint32_t sbb = smem_u32(smem + L::offB + s * L::kB);
+          const uint32_t a_tmem = tmem_base + kAColBase + s * kAStageCols;
+          const uint32_t sbb = smem_u32(smem + kOffTok + s * kTokBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_bf16(d_tmem, smem_desc_k128(sa + kk * 32), smem_desc_k128(sbb + kk * 32), idesc,
-                      (kt | kk) ? 1u : 0u);
+            umma_bf16_ts(d_tmem, a_tmem + kk * 8, smem_desc_k128(sbb + kk * 32), idesc, (kt | kk) ? 1u : 0u);
           umma_commit(&b.empty[s]);
         }
         if (!ok) break;
@@ -269,60 +325,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_bar(&b.drain, 0, lim, abort_flag, a.status, false);
     }
   } else {
-    // epilogue warps 0..3: warp w owns TMEM lanes / tile rows 32w..32w+31
-    const int row_in_tile = warp * 32 + lane;
+    // epilogue warps 0..3: warp w owns TMEM lanes 32w..32w+31 = weight rows of the tile
+    Epi& ep = *reinterpret_cast<Epi*>(smem + kOffEpi);
+    const int n_local = warp * 32 + lane;
     int tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tc) {
       const TileInfo ti = decode_tile(b, a.E, NT, t);
       const int ab = tc & 1;
+      if (!kGateUp) {  // the tile's token metadata, shared by the 4 epilogue warps
+        for (int j = tid; j < kTN; j += 128) {
+          const int pair = j < ti.valid ? a.perm[ti.row0 + j] : 0;
+          ep.pair[ab][j] = pair;
+          ep.w[ab][j] = j < ti.valid ? a.wroute[pair] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.epi_sync[ab]);
+        ok = wait_bar(&b.epi_sync[ab], (tc >> 1) & 1, lim, abort_flag, a.status);
+        if (!ok) break;
+      }
       ok = wait_bar(&b.acc_full[ab], (tc >> 1) & 1, lim, abort_flag, a.status);
       if (!ok) break;
       tc_fence_after();
-      const bool valid = row_in_tile < ti.valid;
-      const int prow = ti.row0 + row_in_tile;
-      const uint16_t* bias = a.bias + (size_t)ti.e * a.N + (size_t)ti.nt * BN;
-      const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + ab * 256;
-      int pair = 0;
-      float wr = 0.f;
-      if (!kGateUp && valid) {
-        pair = a.perm[prow];
-        wr = a.wroute[pair];
-      }
+      const int n = ti.nt * kWM + n_local;
+      const bool valid_n = n < a.N;
+      const float bias = valid_n ? bf16_bits_to_float(a.bias[(size_t)ti.e * a.N + n]) : 0.f;
+      const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + ab * kAccCols;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
+      for (int c0 = 0; c0 < kTN; c0 += 16) {
         uint32_t r[16];
         tmem_ld16(tbase + c0, r);
         tmem_wait_ld();
-        if (valid) {
-          const uint4 bv0 = *reinterpret_cast<const uint4*>(bias + c0);
-          const uint4 bv1 = *reinterpret_cast<const uint4*>(bias + c0 + 8);
-          const uint32_t bw[8] = {bv0.x, bv0.y, bv0.z, bv0.w, bv1.x, bv1.y, bv1.z, bv1.w};
-          if (kGateUp) {
-            uint32_t o[4];
+        if (kGateUp) {
+          // even lanes: gate row n with the up row n+1 of the odd neighbour -> act[token][n/2]
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const float a0 = silu_clamped(__uint_as_float(r[4 * p + 0]) + bf16_bits_to_float(bw[2 * p] & 0xFFFF),
-                                            __uint_as_float(r[4 * p + 1]) + bf16_bits_to_float(bw[2 * p] >> 16));
-              const float a1 =
-                  silu_clamped(__uint_as_float(r[4 * p + 2]) + bf16_bits_to_float(bw[2 * p + 1] & 0xFFFF),
-                               __uint_as_float(r[4 * p + 3]) + bf16_bits_to_float(bw[2 * p + 1] >> 16));
-              o[p] = pack_bf16x2(a0, a1);
-            }
-            const int I = a.N / 2;
-            *reinterpret_cast<uint4*>(a.act_out + (size_t)prow * I + (ti.nt * BN + c0) / 2) =
-                make_uint4(o[0], o[1], o[2], o[3]);
-          } else {
-            float4 y[4];
-            float* yf = reinterpret_cast<float*>(y);
+          for (int j = 0; j < 16; ++j) {
+            const float v = __uint_as_float(r[j]) + bias;
+            const float u = __shfl_xor_sync(0xffffffffu, v, 1);
+            if ((lane & 1) == 0) ep.act[warp][j][lane >> 1] = (uint16_t)float_to_bf16_bits(silu_clamped(v, u));
+          }
+          __syncwarp();
+          // lane L stores 8 outputs (16 bytes) of token c0 + L/2
+          const int j = lane >> 1, part = lane & 1;
+          const int I = a.N / 2;
+          const int i0 = (ti.nt * kWM + warp * 32) / 2 + part * 8;
+          if (c0 + j < ti.valid && i0 < I)
+            *reinterpret_cast<uint4*>(a.act_out + (size_t)(ti.row0 + c0 + j) * I + i0) =
+                *reinterpret_cast<const uint4*>(&ep.act[warp][j][part * 8]);
+          __syncwarp();
+        } else {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const uint32_t bb = (j & 1) ? (bw[j >> 1] >> 16) : (bw[j >> 1] & 0xFFFF);
-              yf[j] = (__uint_as_float(r[j]) + bf16_bits_to_float(bb)) * wr;
-            }
-            float4* dst = reinterpret_cast<float4*>(a.slot_out + (size_t)pair * a.N + ti.nt * BN + c0);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = y[j];
+          for (int j = 0; j < 16; ++j) {
+            const int tok = c0 + j;
+            if (valid_n && tok < ti.valid)
+              a.slot_out[(size_t)ep.pair[ab][tok] * a.N + n] = (__uint_as_float(r[j]) + bias) * ep.w[ab][tok];
           }
         }
       }
@@ -337,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -371,25 +427,26 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool kGateUp>
+template <bool kGateUp>
 cudaError_t launch(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st) {
+  if (a.K % kBK || a.N % 64) return cudaErrorInvalidValue;
   CUtensorMap mapA, mapP;
-  if (!make_map_2d(&mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_ptr, a.K, a.total_rows, kBK, kBM,
+  if (!make_map_2d(&mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_ptr, a.K, a.total_rows, kBK, kTN,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (!make_map_2d(&mapP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.blocks, a.K / 2, (uint64_t)a.E * a.N, kBK / 2, BN,
+  if (!make_map_2d(&mapP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.blocks, a.K / 2, (uint64_t)a.E * a.N, kBK / 2, kWM,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  const size_t smem = smem_total<BN, STAGES>(a.K);
-  auto kern = grouped_mxfp4_gemm<BN, STAGES, kGateUp>;
+  const size_t smem = smem_total(a.K);
+  auto kern = grouped_mxfp4_gemm<kGateUp>;
   static int configured_smem = 0;  // raise the limit only when a larger K needs it
   if ((int)smem > configured_smem) {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     configured_smem = (int)smem;
   }
-  const long long mt_max = ((long long)a.total_rows + kBM - 1) / kBM + a.E;
-  const long long tiles_max = mt_max * (a.N / BN);
+  const long long mt_max = ((long long)a.total_rows + kTN - 1) / kTN + a.E;
+  const long long tiles_max = mt_max * ((a.N + kWM - 1) / kWM);
   const int grid = (int)(tiles_max < sm_count ? tiles_max : sm_count);
   kern<<<grid, kThreads, smem, st>>>(mapA, mapP, a);
   return cudaGetLastError();
@@ -397,30 +454,12 @@ cudaError_t launch(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStrea
 
 }  // namespace
 
-int gemm_pick_bn(int N) {
-  if (N % 240 == 0) return 240;
-  if (N % 192 == 0) return 192;
-  if (N % 128 == 0) return 128;
-  return 64;
-}
-
-template <bool kGateUp>
-cudaError_t launch_dispatch(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st) {
-  if (a.K % kBK || a.N % 64) return cudaErrorInvalidValue;
-  switch (gemm_pick_bn(a.N)) {
-    case 240: return launch<240, 3, kGateUp>(a, a_ptr, sm_count, st);
-    case 192: return launch<192, 4, kGateUp>(a, a_ptr, sm_count, st);
-    case 128: return launch<128, 4, kGateUp>(a, a_ptr, sm_count, st);
-    default: return launch<64, 4, kGateUp>(a, a_ptr, sm_count, st);
-  }
-}
-
 cudaError_t launch_gemm_gateup(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st) {
-  return launch_dispatch<true>(a, a_ptr, sm_count, st);
+  return launch<true>(a, a_ptr, sm_count, st);
 }
 
 cudaError_t launch_gemm_down(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st) {
-  return launch_dispatch<false>(a, a_ptr, sm_count, st);
+  return launch<false>(a, a_ptr, sm_count, st);
 }
 
 }  // namespace moe

@@ -89,6 +89,5 @@ struct GemmArgs {
 // Host: build tensor maps and launch. a_ptr is the bf16 A tensor [total_rows, K].
 cudaError_t launch_gemm_gateup(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st);
 cudaError_t launch_gemm_down(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st);
-int gemm_pick_bn(int N);
 
 }  // namespace moe

@@ -8,47 +8,9 @@
 
 #include <stdint.h>
 
-// Eight consecutive elements (one 32-bit word of packed codes: 4 bytes) with
-// scale byte s -> eight bf16 values, element order preserved (word j of the
-// result holds elements 2j (low half) and 2j+1 (high half)).
-//
-// Exact for 2 <= s <= 252: E2M1 magnitudes have at most two significant bits,
-// so v * 2^(s-127) is a normal bf16. The unscaled bf16 pattern of each code is
-// looked up with byte permutes from two 8-entry tables (low and high byte of
-// the bf16 of |v|), the sign bit is moved into place, and one bf16x2 multiply
-// by 2^(s-127) (exponent field s) applies the scale.
-__device__ __forceinline__ uint4 mx_dequant8_bf16(uint32_t w, uint32_t s) {
-  // |v| for codes 0..7 = 0, .5, 1, 1.5, 2, 3, 4, 6 as bf16: 0000 3F00 3F80 3FC0 4000 4040 4080 40C0
-  constexpr uint32_t kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;  // low bytes of codes 0-3, 4-7
-  constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u;  // high bytes of codes 0-3, 4-7
-  const uint32_t mag = w & 0x77777777u;                       // nibble selectors without sign bits
-  const uint32_t magB = mag >> 16;
-  const uint32_t loA = __byte_perm(kLo0, kLo1, mag), hiA = __byte_perm(kHi0, kHi1, mag);
-  const uint32_t loB = __byte_perm(kLo0, kLo1, magB), hiB = __byte_perm(kHi0, kHi1, magB);
-  uint32_t o0 = __byte_perm(loA, hiA, 0x5140);  // elements 0, 1
-  uint32_t o1 = __byte_perm(loA, hiA, 0x7362);  // elements 2, 3
-  uint32_t o2 = __byte_perm(loB, hiB, 0x5140);  // elements 4, 5
-  uint32_t o3 = __byte_perm(loB, hiB, 0x7362);  // elements 6, 7
-  // Signs: element 2j's sign is bit 8j+3 of w (bit 8j+7 of w<<4) and goes to bit 15;
-  // element 2j+1's sign is bit 8j+7 of w and goes to bit 31.
-  const uint32_t w4 = w << 4;
-  o0 |= __byte_perm(w4, w, 0x4400) & 0x80008000u;
-  o1 |= __byte_perm(w4, w, 0x5511) & 0x80008000u;
-  o2 |= __byte_perm(w4, w, 0x6622) & 0x80008000u;
-  o3 |= __byte_perm(w4, w, 0x7733) & 0x80008000u;
-  const uint32_t sc = s * 0x00800080u;  // bf16x2 (2^(s-127), 2^(s-127))
-  uint4 r;
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r.x) : "r"(o0), "r"(sc));
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r.y) : "r"(o1), "r"(sc));
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r.z) : "r"(o2), "r"(sc));
-  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r.w) : "r"(o3), "r"(sc));
-  return r;
-}
-
 // Four packed bytes -> four f16x2 words of the UNSCALED E2M1 values (exact in
 // f16), with the sm_100a hardware FP4 converter. Word j holds byte j: its low
-// nibble in the low half. The block scale is applied by the caller to fp32
-// partial sums.
+// nibble in the low half.
 __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& h0, uint32_t& h1, uint32_t& h2, uint32_t& h3) {
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
@@ -58,6 +20,50 @@ __device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t& h0, uint32
       "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
       : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
       : "r"(w));
+}
+
+// f16x2 holding E2M1 values (zero or normal f16) -> bf16x2 of the same values
+// times 2^-112: moving the f16 exponent and top mantissa bits down by 3 lands
+// them in the bf16 exponent/mantissa fields (f16 bias 15 vs bf16 bias 127),
+// zeros stay zero, the sign bits are copied. E2M1 values have at most two
+// significant bits, so nothing is lost.
+__device__ __forceinline__ uint32_t f16x2_e2m1_to_bf16x2_m112(uint32_t h) {
+  return ((h & 0x7FFF7FFFu) >> 3) | (h & 0x80008000u);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Eight consecutive elements (one 32-bit word of packed codes: 4 bytes) with
+// scale byte s -> eight bf16 values v * 2^(s-127), element order preserved
+// (word j of the result holds elements 2j (low half) and 2j+1 (high half)).
+//
+// Exact for 2 <= s <= 252: the codes go through the hardware FP4 converter to
+// f16, become bf16 of v * 2^-112 by a bit move, and one bf16x2 multiply by
+// 2^(s-15) (exponent field s+112, representable for s <= 142) applies the
+// scale; for s > 142 a second multiply by 2^(s-142) follows. Every product is
+// a normal bf16 with at most two significant bits, hence exact.
+__device__ __forceinline__ uint4 mx_dequant8_bf16(uint32_t w, uint32_t s) {
+  uint32_t h0, h1, h2, h3;
+  e2m1x8_to_f16x2(w, h0, h1, h2, h3);
+  const uint32_t s1 = s < 142u ? s : 142u;
+  const uint32_t sc = (s1 + 112u) * 0x00800080u;  // bf16x2 (2^(s1-15), 2^(s1-15))
+  uint4 r;
+  r.x = bf16x2_mul(f16x2_e2m1_to_bf16x2_m112(h0), sc);
+  r.y = bf16x2_mul(f16x2_e2m1_to_bf16x2_m112(h1), sc);
+  r.z = bf16x2_mul(f16x2_e2m1_to_bf16x2_m112(h2), sc);
+  r.w = bf16x2_mul(f16x2_e2m1_to_bf16x2_m112(h3), sc);
+  if (s > 142u) {
+    const uint32_t sc2 = (s - 142u + 127u) * 0x00800080u;  // 2^(s-142)
+    r.x = bf16x2_mul(r.x, sc2);
+    r.y = bf16x2_mul(r.y, sc2);
+    r.z = bf16x2_mul(r.z, sc2);
+    r.w = bf16x2_mul(r.w, sc2);
+  }
+  return r;
 }
 
 // acc += a.lo * b.lo + a.hi * b.hi on f16x2 operands with fp32 accumulation
