@@ -351,15 +351,12 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(GemvArgs a) {
 }
 
 cudaError_t configure_gemv(int Cmax) {
-  const int smem = (int)gemv_smem_bytes(Cmax);
-  const int smem_mma = (int)gemv_mma_smem_bytes(Cmax);
-  cudaError_t err = cudaFuncSetAttribute(gemv_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(gemv_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(gemv_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_mma);
-  if (err == cudaSuccess)
-    err = cudaFuncSetAttribute(gemv_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_mma);
+  const size_t smem = gemv_smem_bytes(Cmax);
+  const size_t smem_mma = gemv_mma_smem_bytes(Cmax);
+  cudaError_t err = raise_smem_limit((const void*)gemv_kernel<true>, smem);
+  if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_kernel<false>, smem);
+  if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<true>, smem_mma);
+  if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<false>, smem_mma);
   return err;
 }
 

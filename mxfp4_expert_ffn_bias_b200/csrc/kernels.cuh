@@ -5,6 +5,9 @@
 
 namespace moe {
 
+// Raise (never lower) the dynamic shared memory limit of a kernel.
+cudaError_t raise_smem_limit(const void* func, size_t bytes);
+
 size_t route_smem_bytes(int E);
 constexpr int kRouteTokPerBlock = 32;  // tokens per large-T router block (= one scatter chunk)
 constexpr int kSmallT = 64;            // calls with T <= kSmallT route in one launch

@@ -46,14 +46,26 @@ void free_events(moe_ctx* h) {
   h->ev_slots = h->ev_next = h->ev_count = 0;
 }
 
-// Per-kernel attributes (dynamic shared memory limits), set once per handle.
+}  // namespace
+
+// Raise (never lower) a kernel's dynamic shared memory limit: limits are
+// process-wide per kernel, and other live handles may need a larger one.
+cudaError_t moe::raise_smem_limit(const void* func, size_t bytes) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, func);
+  if (e != cudaSuccess) return e;
+  if ((size_t)fa.maxDynamicSharedSizeBytes >= bytes) return cudaSuccess;
+  return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+namespace {
+
+// Per-kernel attributes (dynamic shared memory limits) for a handle's shapes.
 cudaError_t configure_kernels(const moe_ctx* h) {
   const int T = h->max_T < kSmallT ? h->max_T : kSmallT;
-  cudaError_t e = cudaFuncSetAttribute(route_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)route_small_smem_bytes(T, h->E, h->k, h->HC));
+  cudaError_t e = raise_smem_limit((const void*)route_small_kernel, route_small_smem_bytes(T, h->E, h->k, h->HC));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(route_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)route_smem_bytes(h->E));
+  e = raise_smem_limit((const void*)route_topk_kernel, route_smem_bytes(h->E));
   if (e != cudaSuccess) return e;
   return configure_gemv(h->H > h->I ? h->H : h->I);
 }

@@ -286,3 +286,21 @@ def test_stage_times_reported(moe):
         moe.moe_destroy(h)
     assert n == 3 and len(ms) == 4 and all(m >= 0 for m in ms) and sum(ms) > 0
     assert n2 == 0 and sum(ms2) == 0
+
+
+def test_second_handle_with_smaller_shapes_keeps_first_working(moe):
+    """Kernel launch limits are process-wide: creating a small handle must not break a larger one."""
+    big = CONFIGS["gpt-oss-120b-decode"]
+    inp = inputs_for("gpt-oss-120b-decode")
+    dev = to_device(inp)
+    hb = moe.moe_create(big.H, big.I, big.E, big.k, big.T)
+    hs = moe.moe_create(128, 128, 4, 1, 8)
+    try:
+        out = run_forward(moe, hb, dev, big.T, big.H)
+        torch.cuda.synchronize()
+        assert moe.moe_sync_status(hb) == moe.MOE_OK
+    finally:
+        moe.moe_destroy(hs)
+        moe.moe_destroy(hb)
+    ref, _, _ = oracle.moe_forward(inp, big.k, tokens=[0, 5], threads=NCPU)
+    assert_parity(bf16_dev_to_f64(out)[[0, 5]], ref, "big handle after small handle")
