@@ -117,6 +117,37 @@ moe_status_t moe_forward_hostio(moe_handle_t h, const void* x_host, const float*
                                 const void* gate_up_bias, const uint8_t* down_blocks, const uint8_t* down_scales,
                                 const void* down_bias, int T, void* out_host, void* stream);
 
+/*
+ * The layer for a few tokens WITHOUT any device allocation, for callers that
+ * cannot call cudaMalloc (or an allocating library routine) where they run
+ * the layer: code inside a region that must not allocate or synchronise the
+ * device, allocator callbacks, processes that own no device allocator. The
+ * pages have no counterpart of this entry point; it is a deployment variant
+ * of moe_forward's routed-expert path (same kernels, same results).
+ *
+ * Arguments are moe_forward's, with the shapes given directly instead of a
+ * handle. Limits: T * top_k <= 64, H and I multiples of 64 and <= 4096,
+ * top_k <= 8, top_k <= E <= 256, and the call's scratch must fit the array
+ * (64 routed rows at H = I = 2880 and E = 128 use 1.3 MiB); larger shapes
+ * return MOE_ERR_UNSUPPORTED (use moe_create/moe_forward for them),
+ * malformed ones MOE_ERR_INVALID_ARG.
+ *
+ * Scratch: all intermediate buffers live in one fixed 2 MiB device array
+ * compiled into the library, which every GPU that loads the library holds
+ * until the process exits. The first call on each device looks up that
+ * array's device address (cudaGetSymbolAddress) with the device current; make
+ * that first call before any stream capture. Every call shares the array and
+ * it keeps the previous call's contents (the call clears what must start at
+ * zero itself), so calls that can overlap on the GPU (different streams, or
+ * different host threads without ordering) race on it and must be serialised
+ * by the caller.
+ */
+moe_status_t moe_forward_noalloc(const void* x, const float* router_w, const float* router_b,
+                                 const uint8_t* gate_up_blocks, const uint8_t* gate_up_scales,
+                                 const void* gate_up_bias, const uint8_t* down_blocks, const uint8_t* down_scales,
+                                 const void* down_bias, int H, int I, int E, int top_k, int T, void* out,
+                                 void* stream);
+
 /* Free the handle's workspace. Synchronises the device first. NULL is a no-op. */
 moe_status_t moe_destroy(moe_handle_t h);
 

@@ -5,6 +5,11 @@
 
 namespace moe {
 
+// Enqueue one layer call for a handle whose workspace pointers are already set.
+moe_status_t enqueue_layer(moe_ctx* h, const void* x, const float* rw, const float* rb, const uint8_t* gub,
+                           const uint8_t* gus, const void* gubias, const uint8_t* db, const uint8_t* ds,
+                           const void* dbias, int T, void* out, cudaStream_t st);
+
 // Raise (never lower) the dynamic shared memory limit of a kernel.
 cudaError_t raise_smem_limit(const void* func, size_t bytes);
 

@@ -335,6 +335,14 @@ moe_status_t enqueue_forward(moe_handle_t h, const void* x, const float* rw, con
 
 }  // namespace
 
+// Enqueue one layer call on a handle whose workspace pointers the caller has
+// set up (used by the allocation-free entry point in moe_noalloc.cu).
+moe_status_t moe::enqueue_layer(moe_ctx* h, const void* x, const float* rw, const float* rb, const uint8_t* gub,
+                                const uint8_t* gus, const void* gubias, const uint8_t* db, const uint8_t* ds,
+                                const void* dbias, int T, void* out, cudaStream_t st) {
+  return enqueue_forward(h, x, rw, rb, gub, gus, gubias, db, ds, dbias, T, out, st);
+}
+
 MOE_API moe_status_t moe_forward(moe_handle_t h, const void* x, const float* router_w, const float* router_b,
                                  const uint8_t* gate_up_blocks, const uint8_t* gate_up_scales,
                                  const void* gate_up_bias, const uint8_t* down_blocks, const uint8_t* down_scales,

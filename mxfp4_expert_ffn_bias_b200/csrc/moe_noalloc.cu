@@ -1,0 +1,122 @@
+// moe_forward_noalloc: the layer for a few tokens with no device allocation.
+//
+// For callers that cannot call cudaMalloc (or any allocating library routine)
+// at the point they run the layer: code running where a device allocation is
+// not allowed or not wanted, such as inside a region that must not
+// synchronise the device, a custom allocator's own callback, or a host
+// process that owns no allocator. All scratch memory of the call lives in one
+// file-scope device array of fixed size, so nothing is allocated per call or
+// per handle; the caller passes only its inputs and output.
+//
+// It runs the same kernels as moe_forward's routed-expert (decode) path:
+// one-launch router + top-k + softmax + counting sort, the two warp-MMA GEMVs
+// and the slot combine.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace moe;
+
+namespace {
+
+// Limits of the allocation-free call: T * top_k <= 64 routed rows,
+// H, I <= 4096, E <= 256. The scratch array below holds the largest case.
+constexpr int kNAMaxRows = 64;
+constexpr int kNAMaxHI = 4096;
+constexpr size_t kNAScratchBytes = (size_t)2 << 20;  // 2 MiB per device, held until the process exits
+
+// File-scope scratch of the allocation-free call. In host code this name is a
+// host-side stand-in, not a device address: the address comes from
+// cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNAScratchBytes];
+
+constexpr int kNAMaxDevices = 64;
+std::mutex g_setup_mutex;
+unsigned char* g_scratch_ptr[kNAMaxDevices] = {};
+int g_sm_count[kNAMaxDevices] = {};
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Carve the workspace out of the scratch array; returns the bytes used.
+size_t carve(unsigned char* base, int H, int I, int E, int k, int T, int nHC, Workspace* w) {
+  const size_t Tk = (size_t)T * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    unsigned char* p = base ? base + off : nullptr;
+    off = align256(off + bytes);
+    return p;
+  };
+  w->counts = reinterpret_cast<int*>(take(sizeof(int) * E));
+  w->offsets = reinterpret_cast<int*>(take(sizeof(int) * (E + 1)));
+  w->mt_off = reinterpret_cast<int*>(take(sizeof(int) * (E + 1)));
+  w->touched = reinterpret_cast<int*>(take(sizeof(int) * E));
+  w->n_touched = reinterpret_cast<int*>(take(sizeof(int)));
+  w->idx = reinterpret_cast<int*>(take(sizeof(int) * Tk));
+  w->w = reinterpret_cast<float*>(take(sizeof(float) * Tk));
+  w->perm = reinterpret_cast<int*>(take(sizeof(int) * Tk));
+  w->xexp = reinterpret_cast<int*>(take(sizeof(int) * T));
+  w->act = reinterpret_cast<uint16_t*>(take(sizeof(uint16_t) * Tk * I));
+  w->slot = reinterpret_cast<float*>(take(sizeof(float) * Tk * H));
+  w->status = reinterpret_cast<unsigned*>(take(sizeof(unsigned)));
+  w->partial = reinterpret_cast<float*>(take(sizeof(float) * (size_t)nHC * T * E));
+  w->pmax = reinterpret_cast<float*>(take(sizeof(float) * (size_t)nHC * T));
+  w->ticket = reinterpret_cast<int*>(take(sizeof(int)));
+  return off;
+}
+
+}  // namespace
+
+MOE_API moe_status_t moe_forward_noalloc(const void* x, const float* router_w, const float* router_b,
+                                         const uint8_t* gate_up_blocks, const uint8_t* gate_up_scales,
+                                         const void* gate_up_bias, const uint8_t* down_blocks,
+                                         const uint8_t* down_scales, const void* down_bias, int H, int I, int E,
+                                         int top_k, int T, void* out, void* stream) {
+  const void* ptrs[] = {x,        router_w,    router_b,    gate_up_blocks, gate_up_scales,
+                        gate_up_bias, down_blocks, down_scales, down_bias,  out};
+  for (const void* p : ptrs)
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return MOE_ERR_INVALID_ARG;
+  if (H < 64 || I < 64 || H % 64 || I % 64 || top_k < 1 || top_k > 8 || E < top_k || E > 256 || T < 1)
+    return MOE_ERR_INVALID_ARG;
+  if ((long long)T * top_k > kNAMaxRows || H > kNAMaxHI || I > kNAMaxHI) return MOE_ERR_UNSUPPORTED;
+
+  moe_ctx h;  // a handle on the stack whose workspace points into the scratch array
+  h.H = H;
+  h.I = I;
+  h.E = E;
+  h.k = top_k;
+  h.max_T = T;
+  h.path_opt = 1;  // routed-expert GEMVs
+  h.nHC = 1;
+  for (int n = 1; n <= H / 64; ++n)
+    if ((H / 64) % n == 0 && H / n >= 192) h.nHC = n;
+  h.HC = H / h.nHC;
+  if (carve(nullptr, H, I, E, top_k, T, h.nHC, &h.ws) > kNAScratchBytes) return MOE_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNAMaxDevices) return MOE_ERR_CUDA;
+  {
+    // Once per device, with that device current: the device address of the scratch array.
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (!g_scratch_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return MOE_ERR_CUDA;
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+      g_sm_count[dev] = sms;
+      g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
+    }
+  }
+  h.sm_count = g_sm_count[dev];
+  h.device = dev;
+  carve(g_scratch_ptr[dev], H, I, E, top_k, T, h.nHC, &h.ws);
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (raise_smem_limit((const void*)route_small_kernel, route_small_smem_bytes(T, E, top_k, h.HC)) != cudaSuccess ||
+      configure_gemv(H > I ? H : I) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // The array keeps the previous call's contents: the router's completion ticket must start at zero.
+  if (cudaMemsetAsync(h.ws.ticket, 0, sizeof(int), st) != cudaSuccess) return MOE_ERR_CUDA;
+  return enqueue_layer(&h, x, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks,
+                       down_scales, down_bias, T, out, st);
+}

@@ -48,6 +48,7 @@ SIGNATURES = {
     "moe_create": (_I, [_I, _I, _I, _I, _I, ctypes.POINTER(_P)]),
     "moe_forward": (_I, [_P] * 10 + [_I, _P, _P]),
     "moe_forward_hostio": (_I, [_P] * 10 + [_I, _P, _P]),
+    "moe_forward_noalloc": (_I, [_P] * 9 + [_I, _I, _I, _I, _I, _P, _P]),
     "moe_destroy": (_I, [_P]),
     "moe_status_string": (ctypes.c_char_p, [_I]),
     "moe_set_option": (_I, [_P, _I, ctypes.c_longlong]),
@@ -125,6 +126,15 @@ def moe_forward(h, x, router_w, router_b, gate_up_blocks, gate_up_scales, gate_u
     _check(_lib.moe_forward(h, _ptr(x), _ptr(router_w), _ptr(router_b), _ptr(gate_up_blocks), _ptr(gate_up_scales),
                             _ptr(gate_up_bias), _ptr(down_blocks), _ptr(down_scales), _ptr(down_bias), int(T),
                             _ptr(out), _stream(stream)), "moe_forward")
+
+
+def moe_forward_noalloc(x, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks,
+                        down_scales, down_bias, H: int, I: int, E: int, top_k: int, T: int, out, stream=None) -> None:
+    """The layer for T * top_k <= 64 routed rows without any device allocation (fixed in-library scratch)."""
+    _check(_lib.moe_forward_noalloc(_ptr(x), _ptr(router_w), _ptr(router_b), _ptr(gate_up_blocks),
+                                    _ptr(gate_up_scales), _ptr(gate_up_bias), _ptr(down_blocks), _ptr(down_scales),
+                                    _ptr(down_bias), int(H), int(I), int(E), int(top_k), int(T), _ptr(out),
+                                    _stream(stream)), "moe_forward_noalloc")
 
 
 def moe_forward_hostio(h, x_host: torch.Tensor, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias,
