@@ -55,7 +55,9 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 decode GEMV, 2 grouped GEMM")
-    ap.add_argument("--decode-kernel", type=int, default=1, help="decode GEMV engine: 0 CUDA-core FMA, 1 warp MMA")
+    ap.add_argument("--decode-kernel", type=int, default=-1,
+                    help="decode GEMV engine: 0 CUDA-core FMA, 1 warp MMA per row slab, 2 persistent warp MMA, "
+                         "-1 per stage (gate_up 1, down 2)")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill side measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     return ap.parse_args()
@@ -164,7 +166,7 @@ def weights_list(dev):
                              "down_blocks", "down_scales", "down_bias")]
 
 
-def measure(moe, torch, cfg, dev, T, steps, warmup, path, flush, sampler=None, decode_kernel=1):
+def measure(moe, torch, cfg, dev, T, steps, warmup, path, flush, sampler=None, decode_kernel=-1):
     """Time `steps` layer calls; returns dict with per-step ms list, stage ms (summed), n_touched."""
     h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
     try:
@@ -211,7 +213,7 @@ class _Null:
         return False
 
 
-def measure_e2e(moe, torch, cfg, dev, x_np, T, steps, warmup, path, flush, decode_kernel=1):
+def measure_e2e(moe, torch, cfg, dev, x_np, T, steps, warmup, path, flush, decode_kernel=-1):
     h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
     try:
         moe.moe_set_option(h, moe.MOE_OPT_PATH, path)
@@ -320,7 +322,8 @@ def run_ours(args):
     gu_ms = r["stage_ms"][1]
     if decode:
         achieved = gu_bytes / (gu_ms / 1e3) / 1e9
-        kname = "moe::gemv_mma_kernel<true>" if args.decode_kernel == 1 else "moe::gemv_kernel<true>"
+        kname = {0: "moe::gemv_kernel<true>", 2: "moe::gemv_v_kernel<true>"}.get(args.decode_kernel,
+                                                                            "moe::gemv_mma_kernel<true>")
         roof = {"bound": "hbm", "kernel": f"gate_up GEMV ({kname})", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": None, "peak_kind": f"{peaks_kind} HBM copy bandwidth",

@@ -39,10 +39,45 @@ struct Workspace {
   unsigned* status = nullptr;     // [1] device status word
   float* partial = nullptr;       // [nHC, kSmallT, E] small-T router partial logits
   float* pmax = nullptr;          // [nHC, kSmallT] partial max|x|
-  int* ticket = nullptr;          // [1] small-T router completion counter (0 between calls)
+  float* logits = nullptr;        // [kSmallT, E] small-T router logits
+  uint16_t* w3 = nullptr;         // bf16 [3, E, H] exact three-term split of the router weight (large T)
+  int* ticket = nullptr;          // [kRouteTickets] small-T router completion counters (0 between calls)
   int* chunk_counts = nullptr;    // [nchunk_max, E] pairs per (router chunk, expert)
   int* chunk_base = nullptr;      // [nchunk_max, E] first permuted row per (chunk, expert)
 };
+
+// ------------------------------------------------------------------ host: tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+inline EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major 2-D tensor [outer][inner] of `esize`-byte elements; box of
+// box_outer rows x box_inner elements; out-of-range elements read as zero.
+inline bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t inner,
+                        uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * (uint64_t)esize};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 }  // namespace moe
 
@@ -53,7 +88,7 @@ struct moe_ctx {
   int nHC = 1, HC = 64;  // small-T router: hidden chunks and their width
   int path_opt = 0;
   int decode_max_T = 64;
-  int gemv_variant = 1;
+  int gemv_variant = -1;  // decode GEMV engine; -1: per stage (gate_up 1, down 2)
   long long spin_limit = 2000000;  // microseconds a device-side wait may take before giving up
   moe::Workspace ws;
   cudaStream_t last_stream = nullptr;
@@ -142,6 +177,61 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// ------------------------------------------------------------------ bounded waits
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded, abortable mbarrier wait used by every warp-specialised kernel:
+// gives up after `limit_us` microseconds of wall time (or as soon as another
+// role of the CTA gave up), raising the status word and the CTA's abort flag.
+// With abortable = false (used to drain copies and MMAs still in flight
+// before the CTA exits) only the time limit ends the wait.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, long long limit_us, volatile int* abort_flag,
+                                         unsigned* status, bool abortable = true) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  const uint64_t lim = (uint64_t)limit_us * 1000ull;
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 0) {
+      if (abortable && *abort_flag) return false;
+      if (globaltimer_ns() - t0 > lim) break;
+    }
+  }
+  *abort_flag = 1;
+  atomicOr(status, moe::kStatusTimeout);
+  return false;
+}
+
+// Four 8x8 matrices of 16-bit elements from shared memory: lanes 8i..8i+7
+// give the row addresses (16 bytes each) of matrix i; lane l receives, from
+// each matrix, 32-bit word (l % 4) of row (l / 4).
+__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(saddr));
+}
+
+// 16-byte asynchronous global -> shared copy (L1 bypassed), tracked per thread by commit groups.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's most recent commit groups are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte aligned, bytes % 16 == 0); no completion tracking.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {

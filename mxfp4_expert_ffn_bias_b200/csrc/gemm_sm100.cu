@@ -96,34 +96,6 @@ struct __align__(8) Bars {
 
 size_t smem_total(int K) { return 1024 + kOffSc + 2 * (size_t)kWM * (K / 32) + sizeof(Bars) + 64; }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Bounded, abortable wait used by every role: gives up after `limit_us`
-// microseconds of wall time (or as soon as another role gave up), raising the
-// status word and the CTA's abort flag. With abortable = false (used to drain
-// copies and MMAs still in flight before the CTA exits) only the time limit
-// ends the wait.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, long long limit_us, volatile int* abort_flag,
-                                         unsigned* status, bool abortable = true) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  const uint64_t lim = (uint64_t)limit_us * 1000ull;
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 0) {
-      if (abortable && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > lim) break;
-    }
-  }
-  *abort_flag = 1;
-  atomicOr(status, kStatusTimeout);
-  return false;
-}
-
 struct TileInfo {
   int e, lm, nt, row0, valid;
 };
@@ -398,34 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t inner, uint64_t outer,
-                 uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-  EncodeTiledFn enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * (uint64_t)esize};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  return enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 template <bool kGateUp>
 cudaError_t launch(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st) {

@@ -350,6 +350,414 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(GemvArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- variant 2: warp-private cp.async rings
+//
+// Persistent CTAs (one per SM, 16 warps). A tile is 64 weight rows of one
+// touched expert; CTA c owns a contiguous, balanced range of the
+// n_touched x (R / 64) tiles (mostly one expert, so its tokens are staged
+// once). Warp w takes 16 rows (row group w % 4) and one K quarter (w / 4) of
+// every tile and streams exactly those bytes through its own 4-stage ring in
+// shared memory with 16-byte asynchronous copies (cp.async): a stage is its 16
+// rows x 128 bytes (8 MX blocks), each 128-byte row stored with the XOR
+// swizzle (16-byte unit u of row r at u ^ (r % 8)), so that ldmatrix.x4 reads
+// are conflict-free and hand thread (g, q) word q of the MX block of rows g
+// and g+8: exactly the A fragment layout of the MMA scheme above. Scales and
+// bias of a tile arrive by one bulk copy per pass, issued a pass ahead.
+// Quarters 1..3 hand their partial sums to quarter 0 of the row group through
+// shared memory (an mbarrier hand-off, no CTA-wide wait); quarter 0 adds them
+// in quarter order and runs the epilogue.
+constexpr int kVRows = 64;                     // weight rows per tile
+constexpr int kVQ = 4;                         // K quarters
+constexpr int kVWarps = 4 * kVQ;               // warps per CTA
+constexpr int kVThreads = 32 * kVWarps;
+constexpr int kVChunk = 128;                   // bytes of one row per stage (8 MX blocks)
+constexpr int kVSlot = 16 * kVChunk;           // one warp's stage: 16 rows
+#ifndef MOE_GEMV_STAGES
+#define MOE_GEMV_STAGES 4
+#endif
+constexpr int kVStages = MOE_GEMV_STAGES;      // ring stages per warp
+constexpr int kVPad = 32;                      // f16 padding of a staged token row (conflict-free 16 B loads)
+constexpr int kVMaxE = 256;
+constexpr size_t kSmemLimit = 227 * 1024;
+
+struct __align__(8) GemvBars {
+  uint64_t scf[2];           // scale + bias bytes of a pass landed
+  uint64_t sce[2];           // all warps done with a scale buffer
+  uint64_t red_full[2][4];   // the K quarters 1..3 of a row group left their partial sums
+  uint64_t red_empty[2][4];  // quarter 0 of the row group has read them
+  uint64_t cons;             // CTA-wide barrier, reused by phase
+  int abort_flag;
+};
+
+struct GemvSmem {
+  size_t ring, xs, sc, scb, red, meta, bars, total;
+  int tpp;  // tokens per pass
+};
+
+__host__ __device__ inline GemvSmem gemv_v_layout_tpp(int C, int tpp) {
+  GemvSmem L;
+  const size_t KB = (size_t)(C / 32);
+  L.tpp = tpp;
+  L.ring = 0;
+  L.xs = L.ring + (size_t)kVWarps * kVStages * kVSlot;
+  L.sc = L.xs + (size_t)tpp * (C + kVPad) * 2;
+  L.scb = ((kVRows * KB + 15) / 16) * 16 + kVRows * 2;  // one pass: scales, then the tile's bf16 bias
+  L.red = L.sc + 2 * L.scb;
+  L.meta = L.red + (size_t)2 * (kVQ - 1) * 4 * 8 * 32 * sizeof(float);
+  L.bars = L.meta + (size_t)3 * kVMaxE * 4 + (size_t)2 * 16 * 4;
+  L.total = L.bars + sizeof(GemvBars) + 128;  // + alignment slack of the dynamic buffer
+  return L;
+}
+
+__host__ __device__ inline GemvSmem gemv_v_layout(int C) {
+  const GemvSmem L = gemv_v_layout_tpp(C, 16);
+  return L.total <= kSmemLimit ? L : gemv_v_layout_tpp(C, 8);
+}
+
+size_t gemv_v_smem_bytes(int C) { return gemv_v_layout(C).total; }
+
+// CTA-wide barrier on an mbarrier (bounded, unlike bar.sync, so that a wait
+// that gives up cannot leave the other warps blocked for good).
+__device__ __forceinline__ bool cta_sync(GemvBars& b, uint32_t& phase, long long lim, unsigned* status) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&b.cons);
+  const bool ok = wait_bar(&b.cons, phase, lim, &b.abort_flag, status);
+  phase ^= 1u;
+  return ok;
+}
+
+// One MX block (32 K values) of rows g and g+8 against NT n8 token tiles.
+template <int NT>
+__device__ __forceinline__ void v_block(uint32_t wa, uint32_t wb, const uint16_t* xrow, int CP, uint32_t s0,
+                                        uint32_t s1, float (&acc)[2][4]) {
+  uint32_t f0, f1, f2, f3, f4, f5, f6, f7;
+  e2m1x8_to_f16x2(wa, f0, f1, f2, f3);
+  e2m1x8_to_f16x2(wb, f4, f5, f6, f7);
+  const float sa = __uint_as_float(s0 << 23), sb = __uint_as_float(s1 << 23);
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const uint4 xv = *reinterpret_cast<const uint4*>(xrow + (size_t)nt * 8 * CP);
+    float d0, d1, d2, d3;
+    mma_16816(d0, d1, d2, d3, f0, f4, f1, f5, xv.x, xv.y, 0.f, 0.f, 0.f, 0.f);
+    mma_16816(d0, d1, d2, d3, f2, f6, f3, f7, xv.z, xv.w, d0, d1, d2, d3);
+    acc[nt][0] = fmaf(d0, sa, acc[nt][0]);
+    acc[nt][1] = fmaf(d1, sa, acc[nt][1]);
+    acc[nt][2] = fmaf(d2, sb, acc[nt][2]);
+    acc[nt][3] = fmaf(d3, sb, acc[nt][3]);
+  }
+}
+
+// The blocks [kb0, kb0 + nb) of one stage (nb <= 8; kFull: nb == 8) for this
+// warp's 16 rows. off[p]: this lane's ldmatrix row address for block pair p,
+// relative to the stage.
+template <int NT, bool kFull>
+__device__ __forceinline__ void v_chunk(uint32_t slot, const uint32_t (&off)[4], const uint16_t* xg, int CP,
+                                        const uint8_t* s0, const uint8_t* s1, int kb0, int nb, float (&acc)[2][4]) {
+  const uint16_t* xk = xg + kb0 * 32;
+  const uint8_t* a0 = s0 + kb0;
+  const uint8_t* a1 = s1 + kb0;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    if (kFull || 2 * p < nb) {
+      uint32_t r0, r1, r2, r3;
+      ldmatrix_x4(slot + off[p], r0, r1, r2, r3);
+      v_block<NT>(r0, r1, xk + 64 * p, CP, a0[2 * p], a1[2 * p], acc);
+      if (kFull || 2 * p + 1 < nb) v_block<NT>(r2, r3, xk + 64 * p + 32, CP, a0[2 * p + 1], a1[2 * p + 1], acc);
+    }
+  }
+}
+
+// Position in a CTA's sequence of (tile, token pass, K chunk) steps.
+struct VCursor {
+  long long t;
+  int m0, c;
+  int j, e, r0, Me;
+};
+
+__device__ __forceinline__ void v_cursor_tile(VCursor& u, const int* s_e, const int* s_cnt, int TPE) {
+  u.j = (int)(u.t / TPE);
+  u.e = s_e[u.j];
+  u.r0 = (int)(u.t % TPE) * kVRows;
+  u.Me = s_cnt[u.j];
+}
+
+// Advance by one K chunk (KQ chunks per pass, ceil(Me / tpp) passes per tile).
+__device__ __forceinline__ void v_cursor_step(VCursor& u, int KQ, int tpp, long long t_end, const int* s_e,
+                                              const int* s_cnt, int TPE) {
+  if (++u.c < KQ) return;
+  u.c = 0;
+  u.m0 += tpp;
+  if (u.m0 < u.Me) return;
+  u.m0 = 0;
+  if (++u.t < t_end) v_cursor_tile(u, s_e, s_cnt, TPE);
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kVThreads, 1) gemv_v_kernel(GemvArgs a) {
+  extern __shared__ uint8_t gsm_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 127) & ~uintptr_t(127));
+  const int R = a.R, C = a.C, KB = C / 32, CP = C + kVPad;
+  const int KC = (KB + 7) / 8;          // 8-block chunks of a row
+  const int KQ = (KC + kVQ - 1) / kVQ;  // chunks per K quarter
+  const GemvSmem L = gemv_v_layout(C);
+  const int tpp = L.tpp;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem + L.xs);
+  uint8_t* scs = smem + L.sc;
+  const int scb = (int)L.scb, bias_off = scb - kVRows * 2;
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  int* s_e = reinterpret_cast<int*>(smem + L.meta);  // touched expert j: id, routed rows, first row
+  int* s_cnt = s_e + kVMaxE;
+  int* s_rb = s_cnt + kVMaxE;
+  int* s_pair = s_rb + kVMaxE;                           // staged token m: its (token, slot) pair
+  float* s_scl = reinterpret_cast<float*>(s_pair + 16);  // gate_up: 2^c_t; down: routing weight
+  GemvBars& b = *reinterpret_cast<GemvBars*>(smem + L.bars);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const long long lim = a.spin_limit;
+  const int rgrp = warp & 3, kq = warp >> 2;
+  const int g = lane >> 2, q = lane & 3;
+  const size_t rowbytes = (size_t)KB * 16;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b.scf[i], 1);
+      mbar_init(&b.sce[i], kVWarps);
+      for (int r = 0; r < 4; ++r) {
+        mbar_init(&b.red_full[i][r], kVQ - 1);
+        mbar_init(&b.red_empty[i][r], 1);
+      }
+    }
+    mbar_init(&b.cons, kVWarps);
+    b.abort_flag = 0;
+    fence_barrier_init();
+  }
+  const int n_touched = *a.n_touched;
+  for (int j = tid; j < n_touched; j += kVThreads) {
+    const int e = a.touched[j];
+    s_e[j] = e;
+    s_cnt[j] = a.counts[e];
+    s_rb[j] = a.offsets[e];
+  }
+  __syncthreads();
+
+  const int TPE = R / kVRows;
+  const long long ntiles = (long long)n_touched * TPE;
+  const long long t_begin = ntiles * blockIdx.x / gridDim.x;
+  const long long t_end = ntiles * (blockIdx.x + 1) / gridDim.x;
+  if (t_begin >= t_end) return;
+
+  // scale + bias copies, one pass ahead, by thread 0
+  VCursor sc_cur{t_begin, 0, 0, 0, 0, 0, 0};
+  v_cursor_tile(sc_cur, s_e, s_cnt, TPE);
+  int sc_issued = 0;
+  auto issue_scales = [&]() -> bool {  // thread 0 only
+    if (sc_cur.t >= t_end) return true;
+    const int sb = sc_issued & 1;
+    if (sc_issued >= 2 && !wait_bar(&b.sce[sb], ((sc_issued >> 1) - 1) & 1, lim, &b.abort_flag, a.status))
+      return false;
+    mbar_arrive_expect_tx(&b.scf[sb], kVRows * KB + kVRows * 2);
+    bulk_load(scs + (size_t)sb * scb, a.scales + ((size_t)sc_cur.e * R + sc_cur.r0) * KB, kVRows * KB, &b.scf[sb]);
+    bulk_load(scs + (size_t)sb * scb + bias_off, a.bias + (size_t)sc_cur.e * R + sc_cur.r0, kVRows * 2, &b.scf[sb]);
+    ++sc_issued;
+    sc_cur.c = KQ - 1;  // advance by one whole pass
+    v_cursor_step(sc_cur, KQ, tpp, t_end, s_e, s_cnt, TPE);
+    return true;
+  };
+  bool ok = true;
+  if (tid == 0) ok = issue_scales();
+
+  // weight stream of this warp
+  const uint32_t ring = smem_u32(smem + L.ring) + (uint32_t)warp * kVStages * kVSlot;
+  VCursor ic{t_begin, 0, 0, 0, 0, 0, 0};
+  v_cursor_tile(ic, s_e, s_cnt, TPE);
+  int n_issued = 0;
+  auto issue_chunk = [&]() {  // whole warp; always commits one group
+    if (ic.t < t_end) {
+      const int ch = kq * KQ + ic.c;
+      if (ch < KC) {
+        const int nb = min(8, KB - ch * 8);
+        const uint8_t* src = a.blocks + ((size_t)ic.e * R + ic.r0 + 16 * rgrp) * rowbytes + (size_t)ch * kVChunk;
+        const uint32_t slot = ring + (uint32_t)(n_issued % kVStages) * kVSlot;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int piece = lane + 32 * i, row = piece >> 3, u = piece & 7;
+          if (u < nb) cp_async16(slot + row * kVChunk + ((u ^ (row & 7)) << 4), src + (size_t)row * rowbytes + u * 16);
+        }
+      }
+      v_cursor_step(ic, KQ, tpp, t_end, s_e, s_cnt, TPE);
+    }
+    cp_async_commit();
+    ++n_issued;
+  };
+#pragma unroll 1
+  for (int i = 0; i < kVStages - 1; ++i) issue_chunk();
+
+  uint32_t off[4];
+  {
+    const int m = lane >> 3;                      // matrix this lane addresses
+    const int row = 8 * (m & 1) + (lane & 7);     // row of the stage
+#pragma unroll
+    for (int p = 0; p < 4; ++p) off[p] = (uint32_t)(row * kVChunk + (((2 * p + (m >> 1)) ^ (row & 7)) << 4));
+  }
+  uint32_t cons_ph = 0;
+  int it = 0, pc = 0;
+  int st_e = -1, st_m0 = -1;
+  for (long long t = t_begin; t < t_end && ok; ++t) {
+    const int j = (int)(t / TPE);
+    const int e = s_e[j];
+    const int r0 = (int)(t % TPE) * kVRows;
+    const int Me = s_cnt[j];
+    const int row_base = s_rb[j];
+    for (int m0 = 0; m0 < Me && ok; m0 += tpp, ++pc) {
+      const int mc = min(tpp, Me - m0);
+      if (e != st_e || m0 != st_m0) {  // (re)stage the pass's tokens in f16
+        ok = cta_sync(b, cons_ph, lim, a.status);
+        if (!ok) break;
+        const int nv = C / 8;
+        if (tid < mc) {
+          const int pr = a.perm[row_base + m0 + tid];
+          s_pair[tid] = pr;
+          s_scl[tid] = kGateUp ? exp2_int(a.xexp[pr / a.k]) : a.wroute[pr];
+        }
+        for (int i = tid; i < tpp * nv; i += kVThreads) {
+          const int m = i / nv, c8 = i - m * nv;
+          uint4 v = make_uint4(0, 0, 0, 0);
+          if (m < mc) {
+            if (kGateUp) {  // x * 2^-c_t in f16
+              const int tok = a.perm[row_base + m0 + m] / a.k;
+              const float sc = exp2_int(-a.xexp[tok]);
+              const uint4 raw = reinterpret_cast<const uint4*>(a.xin + (size_t)tok * C)[c8];
+              v.x = pack_f16x2(bf16_bits_to_float(raw.x & 0xFFFF) * sc, bf16_bits_to_float(raw.x >> 16) * sc);
+              v.y = pack_f16x2(bf16_bits_to_float(raw.y & 0xFFFF) * sc, bf16_bits_to_float(raw.y >> 16) * sc);
+              v.z = pack_f16x2(bf16_bits_to_float(raw.z & 0xFFFF) * sc, bf16_bits_to_float(raw.z >> 16) * sc);
+              v.w = pack_f16x2(bf16_bits_to_float(raw.w & 0xFFFF) * sc, bf16_bits_to_float(raw.w >> 16) * sc);
+            } else {
+              v = reinterpret_cast<const uint4*>(a.xin + (size_t)(row_base + m0 + m) * C)[c8];
+            }
+          }
+          reinterpret_cast<uint4*>(xs + (size_t)m * CP)[c8] = v;
+        }
+        ok = cta_sync(b, cons_ph, lim, a.status);
+        if (!ok) break;
+        st_e = e;
+        st_m0 = m0;
+      }
+      if (tid == 0) ok = issue_scales();  // next pass's scales and bias
+      const int sb = pc & 1;
+      ok = ok && wait_bar(&b.scf[sb], (pc >> 1) & 1, lim, &b.abort_flag, a.status);
+      if (!ok) break;
+      const uint8_t* s0 = scs + (size_t)sb * scb + (size_t)(16 * rgrp + g) * KB;
+      const uint8_t* s1 = s0 + 8 * KB;
+      const uint16_t* xg = xs + (size_t)g * CP + 8 * q;
+      const bool two = mc > 8;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int c = 0; c < KQ; ++c, ++it) {
+        issue_chunk();                    // step it + kVStages - 1
+        cp_async_wait<kVStages - 1>();    // this lane's copies of step it landed
+        __syncwarp();                     // ... and every lane's
+        const int ch = kq * KQ + c;
+        if (ch < KC) {
+          const uint32_t slot = ring + (uint32_t)(it % kVStages) * kVSlot;
+          const int kb0 = ch * 8, nb = min(8, KB - kb0);
+          if (nb == 8) {
+            if (two) v_chunk<2, true>(slot, off, xg, CP, s0, s1, kb0, 8, acc);
+            else v_chunk<1, true>(slot, off, xg, CP, s0, s1, kb0, 8, acc);
+          } else {
+            if (two) v_chunk<2, false>(slot, off, xg, CP, s0, s1, kb0, nb, acc);
+            else v_chunk<1, false>(slot, off, xg, CP, s0, s1, kb0, nb, acc);
+          }
+        }
+        __syncwarp();  // the stage is refilled by the next issue
+      }
+      const uint16_t* sbias = reinterpret_cast<const uint16_t*>(scs + (size_t)sb * scb + bias_off);
+      if (kq > 0) {  // hand the partial sums to quarter 0 of the row group; no CTA-wide wait
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.sce[sb]);  // quarter 0 keeps the buffer until its epilogue read the bias
+        if (pc >= 2) ok = wait_bar(&b.red_empty[sb][rgrp], ((pc >> 1) - 1) & 1, lim, &b.abort_flag, a.status);
+        if (!ok) break;
+        float* rd = red + ((size_t)((sb * (kVQ - 1) + kq - 1) * 4 + rgrp) * 8) * 32 + lane;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) rd[(nt * 4 + i) * 32] = acc[nt][i];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&b.red_full[sb][rgrp]);
+        continue;
+      }
+      ok = wait_bar(&b.red_full[sb][rgrp], (pc >> 1) & 1, lim, &b.abort_flag, a.status);
+      if (!ok) break;
+#pragma unroll
+      for (int jq = 0; jq < kVQ - 1; ++jq) {
+        const float* rd = red + ((size_t)((sb * (kVQ - 1) + jq) * 4 + rgrp) * 8) * 32 + lane;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[nt][i] += rd[(nt * 4 + i) * 32];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.red_empty[sb][rgrp]);
+      // acc[nt][0..1]: row r0+16*rgrp+g, tokens nt*8+2q, +1; acc[nt][2..3]: row + 8
+      const int rg = r0 + 16 * rgrp + g;
+      const int lr = 16 * rgrp + g;  // row within the tile
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        if (nt * 8 >= mc) break;  // warp-uniform
+        if (kGateUp) {
+          const float u0 = __shfl_down_sync(0xffffffffu, acc[nt][0], 4);
+          const float u1 = __shfl_down_sync(0xffffffffu, acc[nt][1], 4);
+          const float u2 = __shfl_down_sync(0xffffffffu, acc[nt][2], 4);
+          const float u3 = __shfl_down_sync(0xffffffffu, acc[nt][3], 4);
+          if ((g & 1) == 0) {
+            const int I = R / 2;
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int row = rg + 8 * h2;  // even: gate row; row + 1: up row
+              const float bg = bf16_bits_to_float(sbias[lr + 8 * h2]);
+              const float bu = bf16_bits_to_float(sbias[lr + 8 * h2 + 1]);
+              for (int jj = 0; jj < 2; ++jj) {
+                const int n = nt * 8 + 2 * q + jj;
+                if (n >= mc) continue;
+                const float gacc = h2 ? (jj ? acc[nt][3] : acc[nt][2]) : (jj ? acc[nt][1] : acc[nt][0]);
+                const float uacc = h2 ? (jj ? u3 : u2) : (jj ? u1 : u0);
+                const int prow = row_base + m0 + n;
+                const float sc = s_scl[n];
+                const float gg = fminf(gacc * sc + bg, 7.f);
+                const float uu = fminf(fmaxf(uacc * sc + bu, -7.f), 7.f);
+                const float act = (uu + 1.f) * gg * (1.f / (1.f + expf(-1.702f * gg)));
+                a.act_out[(size_t)prow * I + (row >> 1)] = (uint16_t)(pack_f16x2(act, 0.f) & 0xFFFF);
+              }
+            }
+          }
+        } else {
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int row = rg + 8 * h2;
+            const float bd = bf16_bits_to_float(sbias[lr + 8 * h2]);
+            for (int jj = 0; jj < 2; ++jj) {
+              const int n = nt * 8 + 2 * q + jj;
+              if (n >= mc) continue;
+              const float v = h2 ? (jj ? acc[nt][3] : acc[nt][2]) : (jj ? acc[nt][1] : acc[nt][0]);
+              a.slot_out[(size_t)s_pair[n] * R + row] = (v + bd) * s_scl[n];
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&b.sce[sb]);
+    }
+  }
+  cp_async_wait<0>();  // no copy may land after the CTA has exited
+  if (tid == 0)        // nor a bulk copy of scales issued ahead
+    for (int i = (sc_issued > 2 ? sc_issued - 2 : 0); i < sc_issued; ++i)
+      wait_bar(&b.scf[i & 1], (i >> 1) & 1, lim, &b.abort_flag, a.status, false);
+}
+
+template <bool kGateUp>
+cudaError_t launch_gemv_v(const GemvArgs& a, int sm_count, cudaStream_t st) {
+  if (a.R % kVRows || a.C % 64) return cudaErrorInvalidValue;
+  const size_t smem = gemv_v_smem_bytes(a.C);
+  if (smem > kSmemLimit) return cudaErrorInvalidValue;
+  gemv_v_kernel<kGateUp><<<sm_count, kVThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t configure_gemv(int Cmax) {
   const size_t smem = gemv_smem_bytes(Cmax);
   const size_t smem_mma = gemv_mma_smem_bytes(Cmax);
@@ -357,11 +765,16 @@ cudaError_t configure_gemv(int Cmax) {
   if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_kernel<false>, smem);
   if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<true>, smem_mma);
   if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<false>, smem_mma);
+  const size_t smem_v = gemv_v_smem_bytes(Cmax);
+  if (smem_v <= kSmemLimit) {  // larger rows fall back to variant 1
+    if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_v_kernel<true>, smem_v);
+    if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_v_kernel<false>, smem_v);
+  }
   return err;
 }
 
 cudaError_t launch_gemv_gateup(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st) {
-  (void)sm_count;
+  if (variant == 2 && gemv_v_smem_bytes(a.C) <= kSmemLimit) return launch_gemv_v<true>(a, sm_count, st);
   if (variant == 1) {
     dim3 grid((a.R + kMmaRows - 1) / kMmaRows, max_touched);
     gemv_mma_kernel<true><<<grid, kMmaWarps * 32, gemv_mma_smem_bytes(a.C), st>>>(a);
@@ -373,7 +786,7 @@ cudaError_t launch_gemv_gateup(const GemvArgs& a, int max_touched, int variant, 
 }
 
 cudaError_t launch_gemv_down(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st) {
-  (void)sm_count;
+  if (variant == 2 && gemv_v_smem_bytes(a.C) <= kSmemLimit) return launch_gemv_v<false>(a, sm_count, st);
   if (variant == 1) {
     dim3 grid((a.R + kMmaRows - 1) / kMmaRows, max_touched);
     gemv_mma_kernel<false><<<grid, kMmaWarps * 32, gemv_mma_smem_bytes(a.C), st>>>(a);

@@ -13,7 +13,6 @@ moe_status_t enqueue_layer(moe_ctx* h, const void* x, const float* rw, const flo
 // Raise (never lower) the dynamic shared memory limit of a kernel.
 cudaError_t raise_smem_limit(const void* func, size_t bytes);
 
-size_t route_smem_bytes(int E);
 constexpr int kRouteTokPerBlock = 32;  // tokens per large-T router block (= one scatter chunk)
 constexpr int kSmallT = 64;            // calls with T <= kSmallT route in one launch
 
@@ -33,12 +32,15 @@ struct RouteOut {
 size_t route_small_smem_bytes(int T, int E, int k, int HC);
 __global__ void route_small_kernel(const uint16_t* __restrict__ x, const float* __restrict__ rw,
                                    const float* __restrict__ rb, int T, int H, int E, int k, int HC,
-                                   float* __restrict__ partial, float* __restrict__ pmax, int* __restrict__ ticket,
-                                   RouteOut o);
-__global__ void route_topk_kernel(const uint16_t* __restrict__ x, const float* __restrict__ rw,
-                                  const float* __restrict__ rb, int T, int H, int E, int k, int* __restrict__ idx_out,
-                                  float* __restrict__ w_out, int* __restrict__ counts,
-                                  int* __restrict__ chunk_counts, int* __restrict__ xexp);
+                                   float* __restrict__ partial, float* __restrict__ pmax,
+                                   float* __restrict__ logits, int* __restrict__ ticket, RouteOut o);
+constexpr int kRouteTickets = 1 + 32;  // small-T router: final ticket + one per group of 8 experts (E <= 256)
+__global__ void split_router_kernel(const float* __restrict__ rw, size_t n, uint16_t* __restrict__ w3);
+__global__ void route_mma_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w3,
+                                 const float* __restrict__ rb, int T, int H, int E, int k, int* __restrict__ idx_out,
+                                 float* __restrict__ w_out, int* __restrict__ counts, int* __restrict__ chunk_counts,
+                                 int* __restrict__ xexp);
+size_t route_mma_smem_bytes(int E);
 __global__ void route_scan_kernel(const int* __restrict__ counts, const int* __restrict__ chunk_counts, int nchunk,
                                   int E, int* __restrict__ chunk_base, int* __restrict__ offsets,
                                   int* __restrict__ mt_off, int* __restrict__ touched, int* __restrict__ n_touched);
@@ -67,13 +69,17 @@ struct GemvArgs {
   const float* wroute;     // down: routing weights [T*k]
   uint16_t* act_out;       // gate_up: f16 act [T*k, I]
   float* slot_out;         // down: fp32 [T*k, H] by pair index
-  int R, C, k;
+  unsigned* status;        // device status word (variant 2: a wait that gave up)
+  long long spin_limit;    // microseconds a device-side wait may take (variant 2)
+  int R, C, k, E;
 };
 constexpr int kGemvRows = 64;    // weight rows per block
 constexpr int kGemvTok = 8;      // tokens per pass
 size_t gemv_smem_bytes(int C);
 cudaError_t configure_gemv(int Cmax);
-// variant 0: CUDA-core mixed-precision FMAs; 1: m16n8k16 warp MMAs (same numerics)
+// variant 0: CUDA-core mixed-precision FMAs; 1: m16n8k16 warp MMAs; 2: the same MMAs in persistent CTAs,
+// each warp streaming its rows through its own asynchronous-copy ring (falls back to 1 when its shared
+// memory would exceed the limit). All three have the same numerics.
 cudaError_t launch_gemv_gateup(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st);
 cudaError_t launch_gemv_down(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st);
 

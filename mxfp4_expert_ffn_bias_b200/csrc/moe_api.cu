@@ -30,7 +30,7 @@ cudaError_t alloc(T** p, size_t n) {
 void free_ws(Workspace& w) {
   void* ptrs[] = {w.counts,  w.offsets, w.mt_off,  w.touched, w.n_touched,    w.idx,        w.w,
                   w.perm,    w.xexp,    w.x_perm,  w.act,     w.slot,         w.x_stage,    w.out_stage,
-                  w.status,  w.partial, w.pmax,    w.ticket,  w.chunk_counts, w.chunk_base};
+                  w.status,  w.partial, w.pmax,    w.ticket,  w.chunk_counts, w.chunk_base, w.logits, w.w3};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   w = Workspace{};
@@ -65,7 +65,7 @@ cudaError_t configure_kernels(const moe_ctx* h) {
   const int T = h->max_T < kSmallT ? h->max_T : kSmallT;
   cudaError_t e = raise_smem_limit((const void*)route_small_kernel, route_small_smem_bytes(T, h->E, h->k, h->HC));
   if (e != cudaSuccess) return e;
-  e = raise_smem_limit((const void*)route_topk_kernel, route_smem_bytes(h->E));
+  e = raise_smem_limit((const void*)route_mma_kernel, route_mma_smem_bytes(h->E));
   if (e != cudaSuccess) return e;
   return configure_gemv(h->H > h->I ? h->H : h->I);
 }
@@ -129,7 +129,9 @@ MOE_API moe_status_t moe_create(int H, int I, int E, int top_k, int max_T, moe_h
             alloc(&w.x_stage, (size_t)max_T * H) == cudaSuccess &&
             alloc(&w.out_stage, (size_t)max_T * H) == cudaSuccess && alloc(&w.status, 1) == cudaSuccess &&
             alloc(&w.partial, (size_t)h->nHC * kSmallT * E) == cudaSuccess &&
-            alloc(&w.pmax, (size_t)h->nHC * kSmallT) == cudaSuccess && alloc(&w.ticket, 1) == cudaSuccess &&
+            alloc(&w.pmax, (size_t)h->nHC * kSmallT) == cudaSuccess && alloc(&w.ticket, kRouteTickets) == cudaSuccess &&
+            alloc(&w.logits, (size_t)kSmallT * E) == cudaSuccess &&
+            alloc(&w.w3, (size_t)3 * E * H) == cudaSuccess &&
             alloc(&w.chunk_counts, nchunk * E) == cudaSuccess && alloc(&w.chunk_base, nchunk * E) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();  // clear the allocation error
@@ -137,7 +139,7 @@ MOE_API moe_status_t moe_create(int H, int I, int E, int top_k, int max_T, moe_h
     delete h;
     return MOE_ERR_OOM;
   }
-  if (cudaMemset(w.status, 0, sizeof(unsigned)) != cudaSuccess || cudaMemset(w.ticket, 0, sizeof(int)) != cudaSuccess ||
+  if (cudaMemset(w.status, 0, sizeof(unsigned)) != cudaSuccess || cudaMemset(w.ticket, 0, sizeof(int) * kRouteTickets) != cudaSuccess ||
       configure_kernels(h) != cudaSuccess) {
     free_ws(w);
     delete h;
@@ -172,7 +174,7 @@ MOE_API moe_status_t moe_set_option(moe_handle_t h, int opt, long long v) {
       h->spin_limit = v;
       return MOE_OK;
     case MOE_OPT_DECODE_KERNEL:
-      if (v < 0 || v > 1) return MOE_ERR_INVALID_ARG;
+      if (v < -1 || v > 2) return MOE_ERR_INVALID_ARG;
       h->gemv_variant = (int)v;
       return MOE_OK;
     case MOE_OPT_STAGE_EVENTS: {
@@ -217,7 +219,8 @@ moe_status_t enqueue_route(moe_handle_t h, const void* x, const float* rw, const
     RouteOut o{w.idx, w.w, w.counts, w.offsets, w.mt_off, w.perm, w.touched, w.n_touched, w.xexp};
     dim3 grid((E + 7) / 8, h->nHC);
     route_small_kernel<<<grid, 256, route_small_smem_bytes(T, E, k, h->HC), st>>>(xb, rw, rb, T, H, E, k, h->HC,
-                                                                                 w.partial, w.pmax, w.ticket, o);
+                                                                                 w.partial, w.pmax, w.logits,
+                                                                                 w.ticket, o);
     MOE_CHECK_CUDA(cudaGetLastError());
     if (gather) {
       gather_rows_kernel<<<Tk, 128, 0, st>>>(xb, w.perm, k, H, w.x_perm);
@@ -227,8 +230,13 @@ moe_status_t enqueue_route(moe_handle_t h, const void* x, const float* rw, const
   }
   const int nchunk = (T + kRouteTokPerBlock - 1) / kRouteTokPerBlock;
   MOE_CHECK_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(int) * E, st));
-  route_topk_kernel<<<nchunk, 256, route_smem_bytes(E), st>>>(xb, rw, rb, T, H, E, k, w.idx, w.w, w.counts,
-                                                             w.chunk_counts, w.xexp);
+  {
+    const size_t n = (size_t)E * H;
+    split_router_kernel<<<(int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184), 256, 0, st>>>(rw, n, w.w3);
+    MOE_CHECK_CUDA(cudaGetLastError());
+  }
+  route_mma_kernel<<<nchunk, 256, route_mma_smem_bytes(E), st>>>(xb, w.w3, rb, T, H, E, k, w.idx, w.w, w.counts,
+                                                                w.chunk_counts, w.xexp);
   MOE_CHECK_CUDA(cudaGetLastError());
   route_scan_kernel<<<E, 256, 0, st>>>(w.counts, w.chunk_counts, nchunk, E, w.chunk_base, w.offsets, w.mt_off,
                                        w.touched, w.n_touched);
@@ -266,6 +274,9 @@ moe_status_t enqueue_forward(moe_handle_t h, const void* x, const float* rw, con
     g.n_touched = w.n_touched;
     g.perm = w.perm;
     g.k = k;
+    g.E = E;
+    g.status = w.status;
+    g.spin_limit = h->spin_limit;
     g.blocks = gub;
     g.scales = gus;
     g.bias = static_cast<const uint16_t*>(gubias);
@@ -274,7 +285,7 @@ moe_status_t enqueue_forward(moe_handle_t h, const void* x, const float* rw, con
     g.act_out = w.act;
     g.R = 2 * I;
     g.C = H;
-    MOE_CHECK_CUDA(launch_gemv_gateup(g, max_touched, h->gemv_variant, h->sm_count, st));
+    MOE_CHECK_CUDA(launch_gemv_gateup(g, max_touched, h->gemv_variant < 0 ? 1 : h->gemv_variant, h->sm_count, st));
     if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[2], st));
     g.blocks = db;
     g.scales = ds;
@@ -286,7 +297,7 @@ moe_status_t enqueue_forward(moe_handle_t h, const void* x, const float* rw, con
     g.act_out = nullptr;
     g.R = H;
     g.C = I;
-    MOE_CHECK_CUDA(launch_gemv_down(g, max_touched, h->gemv_variant, h->sm_count, st));
+    MOE_CHECK_CUDA(launch_gemv_down(g, max_touched, h->gemv_variant < 0 ? 2 : h->gemv_variant, h->sm_count, st));
   } else {
     if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[1], st));
     GemmArgs g{};

@@ -61,7 +61,8 @@ size_t carve(unsigned char* base, int H, int I, int E, int k, int T, int nHC, Wo
   w->status = reinterpret_cast<unsigned*>(take(sizeof(unsigned)));
   w->partial = reinterpret_cast<float*>(take(sizeof(float) * (size_t)nHC * T * E));
   w->pmax = reinterpret_cast<float*>(take(sizeof(float) * (size_t)nHC * T));
-  w->ticket = reinterpret_cast<int*>(take(sizeof(int)));
+  w->logits = reinterpret_cast<float*>(take(sizeof(float) * (size_t)T * E));
+  w->ticket = reinterpret_cast<int*>(take(sizeof(int) * kRouteTickets));
   return off;
 }
 
@@ -115,8 +116,8 @@ MOE_API moe_status_t moe_forward_noalloc(const void* x, const float* router_w, c
   if (raise_smem_limit((const void*)route_small_kernel, route_small_smem_bytes(T, E, top_k, h.HC)) != cudaSuccess ||
       configure_gemv(H > I ? H : I) != cudaSuccess)
     return MOE_ERR_CUDA;
-  // The array keeps the previous call's contents: the router's completion ticket must start at zero.
-  if (cudaMemsetAsync(h.ws.ticket, 0, sizeof(int), st) != cudaSuccess) return MOE_ERR_CUDA;
+  // The array keeps the previous call's contents: the router's completion tickets must start at zero.
+  if (cudaMemsetAsync(h.ws.ticket, 0, sizeof(int) * kRouteTickets, st) != cudaSuccess) return MOE_ERR_CUDA;
   return enqueue_layer(&h, x, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias, down_blocks,
                        down_scales, down_bias, T, out, st);
 }

@@ -12,13 +12,9 @@ namespace moe {
 constexpr int kRouteWarps = 8;
 constexpr int kRouteTokPerWarp = 4;
 constexpr int kRouteTok = kRouteWarps * kRouteTokPerWarp;  // tokens per block (== kRouteTokPerBlock)
-constexpr int kRouteHC = 64;                               // hidden columns per staged chunk
 constexpr int kMaxEJ = 8;                                  // experts per lane (E <= 256)
 static_assert(kRouteTok == kRouteTokPerBlock, "router chunk size");
 
-size_t route_smem_bytes(int E) {
-  return sizeof(float) * ((size_t)kRouteTok * kRouteHC + (size_t)E * (kRouteHC + 1)) + sizeof(int) * 256;
-}
 
 // k rounds of a warp-wide arg-max over the logits lg[j] of experts lane + 32j
 // (ties: lower expert index). Every lane ends with the same sele/selv.
@@ -68,91 +64,170 @@ __device__ __forceinline__ int token_exponent(float amax) {
   return max(-100, min(100, c));
 }
 
-// Large-T router: one block handles 32 tokens against all E experts. Logits
-// are fp32 sums over h in increasing order; lane L of a warp owns experts L,
-// L+32, ... The block also counts its own (token, slot) pairs per expert
-// (chunk_counts[block][e]) for the stable scatter that follows.
-__global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(
-    const uint16_t* __restrict__ x, const float* __restrict__ rw, const float* __restrict__ rb, int T, int H,
-    int E, int k, int* __restrict__ idx_out, float* __restrict__ w_out, int* __restrict__ counts,
-    int* __restrict__ chunk_counts, int* __restrict__ xexp) {
+// Large-T router on the tensor cores. The router weight W_r (fp32) is split
+// exactly into three bf16 terms, W_r = W1 + W2 + W3 (W1 = bf16(W_r),
+// W2 = bf16(W_r - W1), W3 = W_r - W1 - W2, each step exact in fp32), so every
+// product x * Wi of a bf16 token is exact and the logits are fp32 sums of the
+// exact products x_h * W_r[e, h], accumulated by m16n8k16 MMAs (the order of
+// the fp32 additions differs from a sequential loop by rounding only).
+__global__ void __launch_bounds__(256) split_router_kernel(const float* __restrict__ rw, size_t n,
+                                                           uint16_t* __restrict__ w3) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const float w = rw[i];
+    const uint32_t b1 = float_to_bf16_bits(w);
+    const float r1 = w - __uint_as_float(b1 << 16);
+    const uint32_t b2 = float_to_bf16_bits(r1);
+    const float r2 = r1 - __uint_as_float(b2 << 16);
+    w3[i] = (uint16_t)b1;
+    w3[n + i] = (uint16_t)b2;
+    w3[2 * n + i] = (uint16_t)float_to_bf16_bits(r2);
+  }
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// max over the eight |bf16| values of a 16-byte vector, as bf16 magnitude bits
+__device__ __forceinline__ uint32_t absmax_bf16x8(uint4 v) {
+  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// One block = 32 tokens (one scatter chunk) x all E experts. Warp w: expert
+// group ng = w % NG (32 experts, four n8 tiles), K group kg = w / NG (every
+// KG-th 32-column chunk of H). Within a 32-column chunk the K order of the two
+// MMAs is permuted identically for tokens and weights: thread (g, q) supplies
+// columns 8q..8q+3 to the first MMA and 8q+4..8q+7 to the second, one 16-byte
+// load per row. K-group partial sums are added in shared memory in kg order.
+// Then, per token, top-k (ties: lower index), softmax over the k, the pair
+// counts per expert and per chunk, and the token's exponent c_t.
+__global__ void __launch_bounds__(256) route_mma_kernel(const uint16_t* __restrict__ x,
+                                                        const uint16_t* __restrict__ w3, const float* __restrict__ rb,
+                                                        int T, int H, int E, int k, int* __restrict__ idx_out,
+                                                        float* __restrict__ w_out, int* __restrict__ counts,
+                                                        int* __restrict__ chunk_counts, int* __restrict__ xexp) {
   extern __shared__ float smem[];
-  float* xs = smem;                               // [kRouteTok][kRouteHC]
-  float* ws = smem + kRouteTok * kRouteHC;        // [E][kRouteHC + 1]
-  int* s_cc = reinterpret_cast<int*>(ws + E * (kRouteHC + 1));  // [E]
+  const int NG = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
+  const int KG = 8 / NG;
+  float* red = smem;                                                 // [KG][32][E]
+  uint32_t* s_amax = reinterpret_cast<uint32_t*>(red + (size_t)KG * 32 * E);  // [KG][32]
+  int* s_cc = reinterpret_cast<int*>(s_amax + KG * 32);             // [E]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, q = lane & 3;
+  const int ng = warp % NG, kg = warp / NG;
   const int t0 = blockIdx.x * kRouteTok;
-  const int EJ = (E + 31) / 32;
   for (int e = tid; e < E; e += blockDim.x) s_cc[e] = 0;
 
-  float acc[kRouteTokPerWarp][kMaxEJ];
+  // token rows of this thread: t0 + 16*mt + g (+8)
+  const uint16_t* xr[4];
+  bool xv[4];
 #pragma unroll
-  for (int i = 0; i < kRouteTokPerWarp; ++i)
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + 16 * (i >> 1) + g + 8 * (i & 1);
+    xv[i] = t < T;
+    xr[i] = x + (size_t)(xv[i] ? t : 0) * H + 8 * q;
+  }
+  const size_t nW = (size_t)E * H;
+  const uint16_t* wr[4];
+  bool wv[4];
 #pragma unroll
-    for (int j = 0; j < kMaxEJ; ++j) acc[i][j] = 0.f;
-  float amax[kRouteTokPerWarp];
+  for (int nt = 0; nt < 4; ++nt) {
+    const int e = 32 * ng + 8 * nt + g;
+    wv[nt] = e < E;
+    wr[nt] = w3 + (size_t)(wv[nt] ? e : 0) * H + 8 * q;
+  }
+  float acc[2][4][4];
 #pragma unroll
-  for (int i = 0; i < kRouteTokPerWarp; ++i) amax[i] = 0.f;
-
-  for (int h0 = 0; h0 < H; h0 += kRouteHC) {
-    for (int i = tid; i < kRouteTok * kRouteHC / 2; i += blockDim.x) {
-      const int tt = i / (kRouteHC / 2), hh = 2 * (i % (kRouteHC / 2));
-      const int t = t0 + tt;
-      uint32_t v = 0;
-      if (t < T) v = *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + hh);
-      xs[tt * kRouteHC + hh] = bf16_bits_to_float(v & 0xFFFF);
-      xs[tt * kRouteHC + hh + 1] = bf16_bits_to_float(v >> 16);
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.f;
+  uint32_t am[4] = {0, 0, 0, 0};
+  const int nK = H / 32;
+  for (int c = kg; c < nK; c += KG) {
+    uint4 a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = xv[i] ? *reinterpret_cast<const uint4*>(xr[i] + 32 * c) : make_uint4(0, 0, 0, 0);
+    if (ng == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) am[i] = max(am[i], absmax_bf16x8(a[i]));
     }
-    for (int i = tid; i < E * kRouteHC / 4; i += blockDim.x) {
-      const int e = i / (kRouteHC / 4), hh = 4 * (i % (kRouteHC / 4));
-      const float4 v = *reinterpret_cast<const float4*>(rw + (size_t)e * H + h0 + hh);
-      float* d = ws + e * (kRouteHC + 1) + hh;
-      d[0] = v.x;
-      d[1] = v.y;
-      d[2] = v.z;
-      d[3] = v.w;
-    }
-    __syncthreads();
 #pragma unroll
-    for (int i = 0; i < kRouteTokPerWarp; ++i) {
-      const float* xr = xs + (warp * kRouteTokPerWarp + i) * kRouteHC;
-      amax[i] = fmaxf(amax[i], fmaxf(fabsf(xr[lane]), fabsf(xr[lane + 32])));
-    }
-#pragma unroll 4
-    for (int hh = 0; hh < kRouteHC; ++hh) {
-      float xv[kRouteTokPerWarp];
+    for (int nt = 0; nt < 4; ++nt) {
+      uint4 bw[3];
 #pragma unroll
-      for (int i = 0; i < kRouteTokPerWarp; ++i) xv[i] = xs[(warp * kRouteTokPerWarp + i) * kRouteHC + hh];
+      for (int sp = 0; sp < 3; ++sp)
+        bw[sp] = wv[nt] ? *reinterpret_cast<const uint4*>(wr[nt] + sp * nW + 32 * c) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int j = 0; j < kMaxEJ; ++j) {
-        if (j < EJ) {
-          const int e = lane + 32 * j;
-          const float wv = (e < E) ? ws[e * (kRouteHC + 1) + hh] : 0.f;
+      for (int mt = 0; mt < 2; ++mt) {
+        const uint4& r0 = a[2 * mt];      // row g
+        const uint4& r1 = a[2 * mt + 1];  // row g + 8
 #pragma unroll
-          for (int i = 0; i < kRouteTokPerWarp; ++i) acc[i][j] = fmaf(xv[i], wv, acc[i][j]);
+        for (int sp = 0; sp < 3; ++sp) {
+          mma_bf16_16816(acc[mt][nt], r0.x, r1.x, r0.y, r1.y, bw[sp].x, bw[sp].y);
+          mma_bf16_16816(acc[mt][nt], r0.z, r1.z, r0.w, r1.w, bw[sp].z, bw[sp].w);
         }
       }
     }
-    __syncthreads();
   }
+  // partial sums of this K group -> red[kg][t][e]
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int e = 32 * ng + 8 * nt + 2 * q;
+      const int tl = 16 * mt + g;
+      if (e < E) {
+        red[((size_t)kg * 32 + tl) * E + e] = acc[mt][nt][0];
+        red[((size_t)kg * 32 + tl + 8) * E + e] = acc[mt][nt][2];
+      }
+      if (e + 1 < E) {
+        red[((size_t)kg * 32 + tl) * E + e + 1] = acc[mt][nt][1];
+        red[((size_t)kg * 32 + tl + 8) * E + e + 1] = acc[mt][nt][3];
+      }
+    }
+  if (ng == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t m = am[i];
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      if (q == 0) s_amax[kg * 32 + 16 * (i >> 1) + g + 8 * (i & 1)] = m;
+    }
+  }
+  __syncthreads();
 
-#pragma unroll
+  // per token: logits, top-k, softmax (warp w: tokens 4w..4w+3)
+  const int EJ = (E + 31) / 32;
+#pragma unroll 1
   for (int i = 0; i < kRouteTokPerWarp; ++i) {
-    const int t = t0 + warp * kRouteTokPerWarp + i;
+    const int tl = warp * kRouteTokPerWarp + i, t = t0 + tl;
     if (t >= T) continue;  // warp-uniform
-    float m = amax[i];
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float lg[kMaxEJ];
 #pragma unroll
     for (int j = 0; j < kMaxEJ; ++j) {
       const int e = lane + 32 * j;
-      lg[j] = (j < EJ && e < E) ? acc[i][j] + rb[e] : -INFINITY;
+      float v = -INFINITY;
+      if (j < EJ && e < E) {
+        v = 0.f;
+        for (int kk = 0; kk < KG; ++kk) v += red[((size_t)kk * 32 + tl) * E + e];
+        v += rb[e];
+      }
+      lg[j] = v;
     }
     int sele[8];
     float selv[8], w[8];
     warp_topk(lg, EJ, E, k, sele, selv);
     if (lane == 0) {
+      uint32_t m = 0;
+      for (int kk = 0; kk < KG; ++kk) m = max(m, s_amax[kk * 32 + tl]);
       softmax_k(selv, k, w);
       for (int s = 0; s < k; ++s) {
         idx_out[t * k + s] = sele[s];
@@ -160,11 +235,17 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_topk_kernel(
         atomicAdd(&counts[sele[s]], 1);  // integer counts: the same whatever the order
         atomicAdd(&s_cc[sele[s]], 1);
       }
-      xexp[t] = token_exponent(m);
+      xexp[t] = token_exponent(bf16_bits_to_float(m));
     }
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) chunk_counts[(size_t)blockIdx.x * E + e] = s_cc[e];
+}
+
+size_t route_mma_smem_bytes(int E) {
+  const int NG = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
+  const int KG = 8 / NG;
+  return sizeof(float) * (size_t)KG * 32 * E + sizeof(uint32_t) * KG * 32 + sizeof(int) * 256;
 }
 
 // ---------------------------------------------------------------- stable counting sort (large T)
@@ -306,13 +387,16 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int* __restric
 
 // ---------------------------------------------------------------- small-T router (one launch)
 
-// For T <= kSmallT. Block (eg, hc) computes partial logits of experts
-// [8*eg, 8*eg+8) over hidden columns [hc*HC, (hc+1)*HC) for every token, and
-// (eg == 0) the partial max|x| of each token. The last block to finish (a
-// ticket counter) sums the partials in hc order, runs top-k and softmax for
-// every token, and performs the stable counting sort of all pairs in shared
-// memory; it then re-arms the ticket. The result does not depend on which
-// block finishes last.
+// For T <= kSmallT, in three phases inside one launch:
+//  1. block (eg, hc) computes the partial logits of experts [8*eg, 8*eg+8)
+//     over hidden columns [hc*HC, (hc+1)*HC) for every token (and, for
+//     eg == 0, the partial max|x| of each token);
+//  2. the last block of expert group eg to finish (a ticket per group) sums
+//     the group's partials in hc order, adds the bias and writes its logits;
+//  3. the last group to finish (a second ticket) runs top-k and softmax for
+//     every token and the stable counting sort of all pairs in shared memory.
+// Each finishing block re-arms its ticket. The result does not depend on
+// which block finishes last.
 size_t route_small_smem_bytes(int T, int E, int k, int HC) {
   const size_t a = ((size_t)T * (HC + 2) * 2 + 15) / 16 * 16 + (size_t)8 * (HC + 1) * 4;
   const size_t b = (size_t)T * E * 4 + (size_t)T * k * 4 + 3 * 260 * 4;
@@ -323,11 +407,11 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
                                                           const float* __restrict__ rw,
                                                           const float* __restrict__ rb, int T, int H, int E, int k,
                                                           int HC, float* __restrict__ partial,
-                                                          float* __restrict__ pmax, int* __restrict__ ticket,
-                                                          RouteOut o) {
+                                                          float* __restrict__ pmax, float* __restrict__ logits,
+                                                          int* __restrict__ ticket, RouteOut o) {
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
-  const int eg = blockIdx.x, hc = blockIdx.y, nHC = gridDim.y;
+  const int eg = blockIdx.x, hc = blockIdx.y, nHC = gridDim.y, nEG = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h0 = hc * HC;
   const int XS = HC + 2, WS = HC + 1;
@@ -343,14 +427,25 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     ws[el * WS + c] = (e < E) ? rw[(size_t)e * H + h0 + c] : 0.f;
   }
   __syncthreads();
-  for (int oi = tid; oi < T * 8; oi += blockDim.x) {
-    const int t = oi >> 3, el = oi & 7, e = eg * 8 + el;
-    if (e >= E) continue;
-    const uint16_t* xr = xs + t * XS;
-    const float* wr = ws + el * WS;
+  // phase 1: outputs (t, el); `tpo` adjacent lanes share one output and split its columns
+  const int nout = T * 8;
+  int tpo = 1;
+  while (tpo < 32 && nout * tpo * 2 <= (int)blockDim.x) tpo *= 2;
+  for (int base = 0; base < nout * tpo; base += blockDim.x) {
+    const int li = base + tid;
+    const int oi = li / tpo, sub = li % tpo;  // tpo divides blockDim.x: a group never straddles two rounds
     float acc = 0.f;
-    for (int c = 0; c < HC; ++c) acc = fmaf(bf16_bits_to_float(xr[c]), wr[c], acc);
-    partial[((size_t)hc * T + t) * E + e] = acc;
+    if (oi < nout) {
+      const int t = oi >> 3, el = oi & 7;
+      const uint16_t* xr = xs + t * XS;
+      const float* wr = ws + el * WS;
+      for (int c = sub; c < HC; c += tpo) acc = fmaf(bf16_bits_to_float(xr[c]), wr[c], acc);
+    }
+    for (int off = tpo >> 1; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (oi < nout && sub == 0) {
+      const int t = oi >> 3, e = eg * 8 + (oi & 7);
+      if (e < E) partial[((size_t)hc * T + t) * E + e] = acc;
+    }
   }
   if (eg == 0) {
     for (int t = warp; t < T; t += 8) {
@@ -364,24 +459,37 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    s_last = atomicAdd(ticket, 1) == (int)(gridDim.x * gridDim.y) - 1;
+    s_last = atomicAdd(&ticket[1 + eg], 1) == nHC - 1;
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
 
-  // ---- last block: logits, top-k, softmax, counting sort
+  // phase 2: the group's logits, partials summed in hc order
+  for (int oi = tid; oi < nout; oi += blockDim.x) {
+    const int t = oi >> 3, e = eg * 8 + (oi & 7);
+    if (e >= E) continue;
+    float v = 0.f;
+    for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
+    logits[(size_t)t * E + e] = v + rb[e];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    ticket[1 + eg] = 0;  // re-arm for the next call
+    __threadfence();
+    s_last = atomicAdd(&ticket[0], 1) == nEG - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  // phase 3 (last group): top-k, softmax, counting sort
   float* lg = reinterpret_cast<float*>(sm);     // [T][E]
   int* s_idx = reinterpret_cast<int*>(lg + (size_t)T * E);  // [T*k]
   int* s_cnt = s_idx + T * k;                   // [E]
   int* s_off = s_cnt + 260;                     // [E+1]
   int* s_mt = s_off + 260;                      // [E+1]
-  for (int i = tid; i < T * E; i += blockDim.x) {
-    const int t = i / E, e = i % E;
-    float v = 0.f;
-    for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
-    lg[i] = v + rb[e];
-  }
+  for (int i = tid; i < T * E; i += blockDim.x) lg[i] = __ldcg(&logits[i]);
   __syncthreads();
   const int EJ = (E + 31) / 32;
   for (int t = warp; t < T; t += 8) {
@@ -394,10 +502,12 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     int sele[8];
     float selv[8], w[8];
     warp_topk(l, EJ, E, k, sele, selv);
+    float m = 0.f;
+    for (int h = lane; h < nHC; h += 32) m = fmaxf(m, __ldcg(&pmax[(size_t)h * T + t]));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (lane == 0) {
       softmax_k(selv, k, w);
-      float m = 0.f;
-      for (int h = 0; h < nHC; ++h) m = fmaxf(m, __ldcg(&pmax[(size_t)h * T + t]));
       o.xexp[t] = token_exponent(m);
       for (int s = 0; s < k; ++s) {
         o.idx[t * k + s] = sele[s];
@@ -426,7 +536,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     for (int j = 0; j < E; ++j)
       if (s_cnt[j] > 0) o.touched[n++] = j;
     *o.n_touched = n;
-    *ticket = 0;  // re-arm for the next call
+    ticket[0] = 0;  // re-arm for the next call
   }
   for (int p = tid; p < Tk; p += blockDim.x) {
     const int e = s_idx[p];

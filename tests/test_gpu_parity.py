@@ -153,8 +153,10 @@ def _run_layer(moe, name_or_cfg, path, T=None, seed=0, tokens=None, repeat=1, va
     return sel, ref, got
 
 
-# (path, decode engine): 1 = routed-expert GEMV (engine 0 CUDA-core FMA, 1 warp MMA), 2 = grouped tcgen05 GEMM
-PATHS = [(1, 0), (1, 1), (2, None)]
+# (path, decode engine): 1 = routed-expert GEMV (engine 0 CUDA-core FMA, 1 warp MMA per slab of rows,
+# 2 warp MMA in persistent CTAs with asynchronous-copy rings, None = the default per-stage choice),
+# 2 = grouped tcgen05 GEMM
+PATHS = [(1, 0), (1, 1), (1, 2), (1, None), (2, None)]
 
 
 @pytest.mark.parametrize("path,variant", PATHS)
@@ -231,7 +233,9 @@ def test_decode_and_prefill_paths_agree(moe):
     a, ref, _ = _run_layer(moe, "gpt-oss-20b-decode", 1)
     b, _, _ = _run_layer(moe, "gpt-oss-20b-decode", 2)
     c, _, _ = _run_layer(moe, "gpt-oss-20b-decode", 1, variant=0)
+    d, _, _ = _run_layer(moe, "gpt-oss-20b-decode", 1, variant=2)
     assert_parity(c, ref, "decode cuda-core engine")
+    assert_parity(d, ref, "decode TMA-fed engine")
     assert_parity(a, ref, "decode")
     assert_parity(b, ref, "prefill")
     s = score(a, b)
