@@ -84,6 +84,33 @@ def gateup_units(cfg, n_touched: int, T: int):
     return bytes_alg, flops
 
 
+# ---------------------------------------------------------------- DRAM traffic of the roofline kernels
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the benchmark's own
+# workload (profiles/ holds the summaries and the commands). A value is reported only while the
+# sources of the kernel's translation unit hash to what they were when it was captured.
+TRAFFIC = {}
+
+
+def _tu_hash(files):
+    import hashlib
+    hsh = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            hsh.update(fh.read())
+    return hsh.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    ent = TRAFFIC.get((kernel, workload))
+    if not ent:
+        return None
+    try:
+        return ent["bytes"] if _tu_hash(ent["files"]) == ent["hash"] else None
+    except OSError:
+        return None
+
+
 # ---------------------------------------------------------------- clocks during the timed region
 
 class ClockSampler:
@@ -167,7 +194,10 @@ def weights_list(dev):
 
 
 def measure(moe, torch, cfg, dev, T, steps, warmup, path, flush, sampler=None, decode_kernel=-1):
-    """Time `steps` layer calls; returns dict with per-step ms list, stage ms (summed), n_touched."""
+    """Time `steps` layer calls, each bracketed by its own CUDA events (the headline window), then
+    `steps` more calls with CUDA events also between the stages (the per-stage window: events between
+    kernels stop consecutive kernels from overlapping their launch, so they stay out of the headline).
+    Returns the per-step ms of the first window, the average stage ms of the second and n_touched."""
     h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
     try:
         moe.moe_set_option(h, moe.MOE_OPT_PATH, path)
@@ -183,7 +213,6 @@ def measure(moe, torch, cfg, dev, T, steps, warmup, path, flush, sampler=None, d
         moe.moe_debug_route(h, dev["x"], dev["router_w"], dev["router_b"], T, idx)
         torch.cuda.synchronize()
         n_touched = int(torch.unique(idx).numel())
-        moe.moe_set_option(h, moe.MOE_OPT_STAGE_EVENTS, steps)
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         torch.cuda.synchronize()
         ctx = sampler if sampler is not None else _Null()
@@ -195,6 +224,11 @@ def measure(moe, torch, cfg, dev, T, steps, warmup, path, flush, sampler=None, d
                 evs[i][1].record(st)
             torch.cuda.synchronize()
         step_ms = [a.elapsed_time(b) for a, b in evs]
+        moe.moe_set_option(h, moe.MOE_OPT_STAGE_EVENTS, steps)
+        for i in range(steps):
+            flush.zero_()
+            moe.moe_forward(h, dev["x"], *W, T, out)
+        torch.cuda.synchronize()
         stage_ms, ncalls = moe.moe_stage_times(h)
         status = moe.moe_sync_status(h)
         if status != moe.MOE_OK:
@@ -259,7 +293,7 @@ def cpu_baseline(cfg, inputs, budget_s=10.0):
 
 def launches_per_call(T: int, decode: bool) -> int:
     """Kernels of ours per layer call (memset nodes not counted)."""
-    route = 1 if T <= 64 else 3  # one fused router, or router + scan + scatter
+    route = 1 if T <= 64 else 4  # one fused router, or weight split + router + scan + scatter
     if decode:
         return route + 3  # gate_up GEMV, down GEMV, combine
     gather = 1 if T <= 64 else 0  # the large-T scatter gathers rows itself
@@ -326,14 +360,17 @@ def run_ours(args):
                                                                             "moe::gemv_mma_kernel<true>")
         roof = {"bound": "hbm", "kernel": f"gate_up GEMV ({kname})", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "peak_kind": f"{peaks_kind} HBM copy bandwidth",
+                "traffic": traffic_for(kname, cfg.name), "peak_kind": f"{peaks_kind} HBM copy bandwidth",
                 "algorithmic_bytes_per_launch": gu_bytes}
     else:
         achieved = gu_flops / (gu_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "kernel": "gate_up grouped GEMM (moe::grouped_mxfp4_gemm<.., true>)",
+        kname = "moe::grouped_mxfp4_gemm<true>"
+        roof = {"bound": "tensor", "kernel": f"gate_up grouped GEMM ({kname})",
                 "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic_for(kname, cfg.name),
                 "peak_kind": f"{peaks_kind} dense bf16 (burst)", "algorithmic_flops_per_launch": gu_flops}
+    roof["window"] = ("kernel time from CUDA events around the stage, over a second window of the same number "
+                      "of steps right after the headline window")
     layer_gbs = bytes_alg / (ms_step / 1e3) / 1e9
     layer_tflops = flops_alg / (ms_step / 1e3) / 1e12
     line = {

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe.h"
 
 #define MOE_API extern "C" __attribute__((visibility("default")))
@@ -45,6 +47,27 @@ struct Workspace {
   int* chunk_counts = nullptr;    // [nchunk_max, E] pairs per (router chunk, expert)
   int* chunk_base = nullptr;      // [nchunk_max, E] first permuted row per (chunk, expert)
 };
+
+// ------------------------------------------------------------------ host: launches
+
+// Launch with programmatic dependent launch allowed: the kernel may be scheduled
+// while the previous kernel of the stream finishes; every kernel of the layer
+// starts with pdl_wait(), which returns once that kernel has completed and its
+// memory is visible, so stream order is kept for all global-memory effects.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ------------------------------------------------------------------ host: tensor maps
 
@@ -177,6 +200,15 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Wait until the previous kernel of the stream has completed (no-op without PDL),
+// then let the next kernel of the stream be scheduled.
+__device__ __forceinline__ void pdl_wait_and_trigger() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ------------------------------------------------------------------ bounded waits

@@ -129,6 +129,7 @@ template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_mxfp4_gemm(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapP,
                        GemmArgs a) {
+  pdl_wait_and_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int KB = a.K / 32;
@@ -392,7 +393,10 @@ cudaError_t launch(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStrea
   const long long mt_max = ((long long)a.total_rows + kTN - 1) / kTN + a.E;
   const long long tiles_max = mt_max * ((a.N + kWM - 1) / kWM);
   const int grid = (int)(tiles_max < sm_count ? tiles_max : sm_count);
-  kern<<<grid, kThreads, smem, st>>>(mapA, mapP, a);
+  {
+    const cudaError_t e_ = launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, mapA, mapP, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 

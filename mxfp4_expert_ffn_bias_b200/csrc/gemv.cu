@@ -37,6 +37,7 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 
 template <bool kGateUp>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
+  pdl_wait_and_trigger();
   extern __shared__ __align__(16) uint16_t xs[];  // f16 [kGemvTok][C]
   const int slotj = blockIdx.y;
   if (slotj >= *a.n_touched) return;
@@ -241,6 +242,7 @@ __device__ __forceinline__ void mma_compute(const MmaGroup& G, int b0, int KB, b
 // (8 x C, rows padded by 16 bytes) and the block's scale bytes.
 template <bool kGateUp>
 __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(GemvArgs a) {
+  pdl_wait_and_trigger();
   extern __shared__ __align__(16) uint8_t gsm[];
   const int slotj = blockIdx.y;
   if (slotj >= *a.n_touched) return;
@@ -494,6 +496,7 @@ __device__ __forceinline__ void v_cursor_step(VCursor& u, int KQ, int tpp, long 
 
 template <bool kGateUp>
 __global__ void __launch_bounds__(kVThreads, 1) gemv_v_kernel(GemvArgs a) {
+  pdl_wait_and_trigger();
   extern __shared__ uint8_t gsm_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 127) & ~uintptr_t(127));
   const int R = a.R, C = a.C, KB = C / 32, CP = C + kVPad;
@@ -754,7 +757,10 @@ cudaError_t launch_gemv_v(const GemvArgs& a, int sm_count, cudaStream_t st) {
   if (a.R % kVRows || a.C % 64) return cudaErrorInvalidValue;
   const size_t smem = gemv_v_smem_bytes(a.C);
   if (smem > kSmemLimit) return cudaErrorInvalidValue;
-  gemv_v_kernel<kGateUp><<<sm_count, kVThreads, smem, st>>>(a);
+  {
+    const cudaError_t e_ = launch_pdl(gemv_v_kernel<kGateUp>, dim3(sm_count), dim3(kVThreads), smem, st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   return cudaGetLastError();
 }
 
@@ -777,10 +783,17 @@ cudaError_t launch_gemv_gateup(const GemvArgs& a, int max_touched, int variant, 
   if (variant == 2 && gemv_v_smem_bytes(a.C) <= kSmemLimit) return launch_gemv_v<true>(a, sm_count, st);
   if (variant == 1) {
     dim3 grid((a.R + kMmaRows - 1) / kMmaRows, max_touched);
-    gemv_mma_kernel<true><<<grid, kMmaWarps * 32, gemv_mma_smem_bytes(a.C), st>>>(a);
+    {
+    const cudaError_t e_ =
+        launch_pdl(gemv_mma_kernel<true>, grid, dim3(kMmaWarps * 32), gemv_mma_smem_bytes(a.C), st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   } else {
     dim3 grid(a.R / kGemvRows, max_touched);
-    gemv_kernel<true><<<grid, kGemvThreads, gemv_smem_bytes(a.C), st>>>(a);
+    {
+    const cudaError_t e_ = launch_pdl(gemv_kernel<true>, grid, dim3(kGemvThreads), gemv_smem_bytes(a.C), st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   }
   return cudaGetLastError();
 }
@@ -789,10 +802,17 @@ cudaError_t launch_gemv_down(const GemvArgs& a, int max_touched, int variant, in
   if (variant == 2 && gemv_v_smem_bytes(a.C) <= kSmemLimit) return launch_gemv_v<false>(a, sm_count, st);
   if (variant == 1) {
     dim3 grid((a.R + kMmaRows - 1) / kMmaRows, max_touched);
-    gemv_mma_kernel<false><<<grid, kMmaWarps * 32, gemv_mma_smem_bytes(a.C), st>>>(a);
+    {
+    const cudaError_t e_ =
+        launch_pdl(gemv_mma_kernel<false>, grid, dim3(kMmaWarps * 32), gemv_mma_smem_bytes(a.C), st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   } else {
     dim3 grid(a.R / kGemvRows, max_touched);
-    gemv_kernel<false><<<grid, kGemvThreads, gemv_smem_bytes(a.C), st>>>(a);
+    {
+    const cudaError_t e_ = launch_pdl(gemv_kernel<false>, grid, dim3(kGemvThreads), gemv_smem_bytes(a.C), st, a);
+    if (e_ != cudaSuccess) return e_;
+  }
   }
   return cudaGetLastError();
 }

@@ -218,12 +218,11 @@ moe_status_t enqueue_route(moe_handle_t h, const void* x, const float* rw, const
   if (T <= kSmallT) {
     RouteOut o{w.idx, w.w, w.counts, w.offsets, w.mt_off, w.perm, w.touched, w.n_touched, w.xexp};
     dim3 grid((E + 7) / 8, h->nHC);
-    route_small_kernel<<<grid, 256, route_small_smem_bytes(T, E, k, h->HC), st>>>(xb, rw, rb, T, H, E, k, h->HC,
-                                                                                 w.partial, w.pmax, w.logits,
-                                                                                 w.ticket, o);
+    MOE_CHECK_CUDA(launch_pdl(route_small_kernel, grid, dim3(256), route_small_smem_bytes(T, E, k, h->HC), st, xb,
+                              rw, rb, T, H, E, k, h->HC, w.partial, w.pmax, w.logits, w.ticket, o));
     MOE_CHECK_CUDA(cudaGetLastError());
     if (gather) {
-      gather_rows_kernel<<<Tk, 128, 0, st>>>(xb, w.perm, k, H, w.x_perm);
+      MOE_CHECK_CUDA(launch_pdl(gather_rows_kernel, dim3(Tk), dim3(128), 0, st, xb, w.perm, k, H, w.x_perm));
       MOE_CHECK_CUDA(cudaGetLastError());
     }
     return MOE_OK;
@@ -232,17 +231,18 @@ moe_status_t enqueue_route(moe_handle_t h, const void* x, const float* rw, const
   MOE_CHECK_CUDA(cudaMemsetAsync(w.counts, 0, sizeof(int) * E, st));
   {
     const size_t n = (size_t)E * H;
-    split_router_kernel<<<(int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184), 256, 0, st>>>(rw, n, w.w3);
+    const int nb = (int)((n + 255) / 256 < 1184 ? (n + 255) / 256 : 1184);
+    MOE_CHECK_CUDA(launch_pdl(split_router_kernel, dim3(nb), dim3(256), 0, st, rw, n, w.w3));
     MOE_CHECK_CUDA(cudaGetLastError());
   }
-  route_mma_kernel<<<nchunk, 256, route_mma_smem_bytes(E), st>>>(xb, w.w3, rb, T, H, E, k, w.idx, w.w, w.counts,
-                                                                w.chunk_counts, w.xexp);
+  MOE_CHECK_CUDA(launch_pdl(route_mma_kernel, dim3(nchunk), dim3(256), route_mma_smem_bytes(E), st, xb, w.w3, rb, T, H,
+                            E, k, w.idx, w.w, w.counts, w.chunk_counts, w.xexp));
   MOE_CHECK_CUDA(cudaGetLastError());
-  route_scan_kernel<<<E, 256, 0, st>>>(w.counts, w.chunk_counts, nchunk, E, w.chunk_base, w.offsets, w.mt_off,
-                                       w.touched, w.n_touched);
+  MOE_CHECK_CUDA(launch_pdl(route_scan_kernel, dim3(E), dim3(256), 0, st, w.counts, w.chunk_counts, nchunk, E,
+                            w.chunk_base, w.offsets, w.mt_off, w.touched, w.n_touched));
   MOE_CHECK_CUDA(cudaGetLastError());
-  route_scatter_kernel<<<nchunk, 256, 0, st>>>(w.idx, w.chunk_base, T, E, k, xb, H, gather ? 1 : 0, w.perm,
-                                               w.x_perm);
+  MOE_CHECK_CUDA(launch_pdl(route_scatter_kernel, dim3(nchunk), dim3(256), 0, st, w.idx, w.chunk_base, T, E, k, xb,
+                            H, gather ? 1 : 0, w.perm, w.x_perm));
   MOE_CHECK_CUDA(cudaGetLastError());
   return MOE_OK;
 }
@@ -334,7 +334,8 @@ moe_status_t enqueue_forward(moe_handle_t h, const void* x, const float* rw, con
   int blocks = (int)((n4 + threads - 1) / threads);
   const int cap = h->sm_count * 8;
   if (blocks > cap) blocks = cap;
-  combine_kernel<<<blocks, threads, 0, st>>>(w.slot, T, H, k, static_cast<uint16_t*>(out));
+  MOE_CHECK_CUDA(launch_pdl(combine_kernel, dim3(blocks), dim3(threads), 0, st, w.slot, T, H, k,
+                            static_cast<uint16_t*>(out)));
   MOE_CHECK_CUDA(cudaGetLastError());
   if (rec) {
     MOE_CHECK_CUDA(cudaEventRecord(ev[4], st));

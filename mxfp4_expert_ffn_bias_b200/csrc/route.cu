@@ -72,6 +72,7 @@ __device__ __forceinline__ int token_exponent(float amax) {
 // the fp32 additions differs from a sequential loop by rounding only).
 __global__ void __launch_bounds__(256) split_router_kernel(const float* __restrict__ rw, size_t n,
                                                            uint16_t* __restrict__ w3) {
+  pdl_wait_and_trigger();
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
     const float w = rw[i];
     const uint32_t b1 = float_to_bf16_bits(w);
@@ -112,6 +113,7 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const uint16_t* __restri
                                                         int T, int H, int E, int k, int* __restrict__ idx_out,
                                                         float* __restrict__ w_out, int* __restrict__ counts,
                                                         int* __restrict__ chunk_counts, int* __restrict__ xexp) {
+  pdl_wait_and_trigger();
   extern __shared__ float smem[];
   const int NG = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
   const int KG = 8 / NG;
@@ -300,6 +302,7 @@ __global__ void __launch_bounds__(256) route_scan_kernel(const int* __restrict__
                                                          int* __restrict__ chunk_base, int* __restrict__ offsets,
                                                          int* __restrict__ mt_off, int* __restrict__ touched,
                                                          int* __restrict__ n_touched) {
+  pdl_wait_and_trigger();
   __shared__ int s_off[257], s_mt[257], s_part[256];
   const int e = blockIdx.x, tid = threadIdx.x;
   prefix_counts(counts, E, s_off, s_mt);
@@ -359,6 +362,7 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int* __restric
                                                             const int* __restrict__ chunk_base, int T, int E, int k,
                                                             const uint16_t* __restrict__ x, int H, int gather,
                                                             int* __restrict__ perm, uint16_t* __restrict__ x_perm) {
+  pdl_wait_and_trigger();
   __shared__ int s_idx[kRouteTok * 8], s_dest[kRouteTok * 8];
   const int b = blockIdx.x, tid = threadIdx.x;
   const int t0 = b * kRouteTok;
@@ -409,6 +413,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
                                                           int HC, float* __restrict__ partial,
                                                           float* __restrict__ pmax, float* __restrict__ logits,
                                                           int* __restrict__ ticket, RouteOut o) {
+  pdl_wait_and_trigger();
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
   const int eg = blockIdx.x, hc = blockIdx.y, nHC = gridDim.y, nEG = gridDim.x;
@@ -417,11 +422,14 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
   const int XS = HC + 2, WS = HC + 1;
   uint16_t* xs = reinterpret_cast<uint16_t*>(sm);
   float* ws = reinterpret_cast<float*>(sm + ((size_t)T * XS * 2 + 15) / 16 * 16);
+  // (unrolled so that the loads of several iterations are in flight together)
+#pragma unroll 8
   for (int i = tid; i < T * (HC / 2); i += blockDim.x) {
     const int t = i / (HC / 2), c2 = i % (HC / 2);
     *reinterpret_cast<uint32_t*>(xs + t * XS + 2 * c2) =
         *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + 2 * c2);
   }
+#pragma unroll 8
   for (int i = tid; i < 8 * HC; i += blockDim.x) {
     const int el = i / HC, c = i % HC, e = eg * 8 + el;
     ws[el * WS + c] = (e < E) ? rw[(size_t)e * H + h0 + c] : 0.f;
@@ -470,6 +478,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     const int t = oi >> 3, e = eg * 8 + (oi & 7);
     if (e >= E) continue;
     float v = 0.f;
+#pragma unroll 8
     for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
     logits[(size_t)t * E + e] = v + rb[e];
   }
@@ -489,6 +498,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
   int* s_cnt = s_idx + T * k;                   // [E]
   int* s_off = s_cnt + 260;                     // [E+1]
   int* s_mt = s_off + 260;                      // [E+1]
+#pragma unroll 8
   for (int i = tid; i < T * E; i += blockDim.x) lg[i] = __ldcg(&logits[i]);
   __syncthreads();
   const int EJ = (E + 31) / 32;
@@ -549,6 +559,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
 // x_perm[p] = x[perm[p] / k]: one block per permuted row, 16-byte vectors.
 __global__ void __launch_bounds__(128) gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ perm,
                                                           int k, int H, uint16_t* __restrict__ x_perm) {
+  pdl_wait_and_trigger();
   const int p = blockIdx.x;
   const int t = perm[p] / k;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -559,6 +570,7 @@ __global__ void __launch_bounds__(128) gather_rows_kernel(const uint16_t* __rest
 // out[t, j] = bf16( sum_{s=0..k-1} slot[t*k+s, j] ), summed in slot order.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ slot, int T, int H, int k,
                                                       uint16_t* __restrict__ out) {
+  pdl_wait_and_trigger();
   const int H4 = H / 4;
   const long long n = (long long)T * H4;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
