@@ -69,6 +69,27 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// As launch_pdl, as one cluster of `cluster_x` CTAs along x per `cluster_x` blocks of the grid.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------------ host: tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -112,6 +133,7 @@ struct moe_ctx {
   int path_opt = 0;
   int decode_max_T = 64;
   int gemv_variant = -1;  // decode GEMV engine; -1: per stage (gate_up 1, down 2)
+  int cluster_cs = 0;     // small-T router on one cluster of this many CTAs (0: the three-phase router)
   long long spin_limit = 2000000;  // microseconds a device-side wait may take before giving up
   moe::Workspace ws;
   cudaStream_t last_stream = nullptr;
@@ -180,6 +202,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, letting the thread sleep up to `ns` nanoseconds for the phase to complete.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -230,8 +263,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, long lo
   const uint64_t t0 = globaltimer_ns();
   const uint64_t lim = (uint64_t)limit_us * 1000ull;
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255) == 0) {
+    // sleep in the barrier (up to 20 us per try) instead of spinning: waiting warps take no issue slots
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if ((i & 15) == 0) {
       if (abortable && *abort_flag) return false;
       if (globaltimer_ns() - t0 > lim) break;
     }

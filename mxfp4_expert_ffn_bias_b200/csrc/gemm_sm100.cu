@@ -17,14 +17,16 @@
 // Per CTA (one per SM), warp-specialised:
 //   warp 4      TMA producer: token tile (192 x 64 bf16, 128B swizzle) and the
 //               packed weight tile (128 x 32 bytes) per K step into a ring of
-//               4 shared-memory stages; the tile's E8M0 scales (128 x K/32
+//               6 shared-memory stages; the tile's E8M0 scales (128 x K/32
 //               bytes, contiguous) with one bulk copy per output tile.
 //   warps 6..   dequant (8 warps): warp w converts part (w-6)/4 of each K step
-//               for TMEM sub-partition w % 4 (lanes = weight rows); converting
-//               step k+1 overlaps the TMEM store of step k.
-//   warp 5      one thread issues 4 MMAs (K = 16 each) per stage, commits to
-//               free the stage and, after the last K step, hands the
-//               accumulator to the epilogue.
+//               for TMEM sub-partition w % 4 (lanes = weight rows) into a ring
+//               of 4 TMEM A stages, handing each stage over as soon as it is
+//               written; the deeper shared-memory ring keeps the next steps'
+//               bytes landed ahead of the conversion.
+//   warp 5      one thread issues 4 MMAs (K = 16 each) per step, commits to
+//               free the shared-memory and TMEM stages and, after the last K
+//               step, hands the accumulator to the epilogue.
 //   warps 0-3   epilogue: tcgen05.ld (lane = weight row, column = token), add
 //               the bias and either
 //                 gate_up: pair gate row 2i with up row 2i+1 (adjacent lanes;
@@ -48,7 +50,11 @@ namespace {
 
 constexpr int kWM = 128;                    // weight rows per tile (MMA M, TMEM lanes)
 constexpr int kTN = kBM;                    // token rows per tile (MMA N)
-constexpr int kStages = 4;
+#ifndef MOE_GEMM_STAGES
+#define MOE_GEMM_STAGES 6
+#endif
+constexpr int kStages = MOE_GEMM_STAGES;    // TMA ring (token + packed tiles) in shared memory
+constexpr int kTStages = 4;                 // TMEM ring of dequantised A stages
 #ifndef MOE_DEQ_WARPS
 #define MOE_DEQ_WARPS 8  // measured: 8 (900 us) beat 16 (972 us) on the 20b prefill gate_up
 #endif
@@ -62,11 +68,11 @@ constexpr int kAccCols = kTN;               // fp32 columns of one accumulator
 constexpr int kAStageCols = kBK / 2;        // TMEM columns of one bf16 A stage (64 K values)
 constexpr int kAColBase = 2 * kAccCols;     // A stages follow the two accumulators
 constexpr int kTmemCols = 512;
-static_assert(kAColBase + kStages * kAStageCols <= kTmemCols, "TMEM budget");
+static_assert(kAColBase + kTStages * kAStageCols <= kTmemCols, "TMEM budget");
 constexpr int kMaxE = 256;
 
 constexpr int kTokBytes = kTN * 128;        // one token stage (64 bf16 per row)
-constexpr int kPackBytes = kWM * 32;        // one packed weight stage (32 bytes per row)
+constexpr int kPackBytes = kWM * 32;        // one packed weight stage: two halves [2][kWM rows][16 bytes]
 constexpr int kOffTok = 0;
 constexpr int kOffPack = kOffTok + kStages * kTokBytes;
 constexpr int kOffEpi = kOffPack + kStages * kPackBytes;  // epilogue staging (see Epi)
@@ -79,8 +85,9 @@ constexpr int kOffSc = kOffEpi + (int)((sizeof(Epi) + 127) / 128 * 128);  // 2 s
 
 struct __align__(8) Bars {
   uint64_t full_ab[kStages];   // TMA landed (token + packed tiles)
-  uint64_t full_b[kStages];    // TMEM A stage written by the dequant warps
-  uint64_t empty[kStages];     // MMAs of the stage done
+  uint64_t empty[kStages];     // MMAs of the step done (shared-memory stage free)
+  uint64_t full_b[kTStages];   // TMEM A stage written by the dequant warps
+  uint64_t tfree[kTStages];    // MMAs that read the TMEM A stage done
   uint64_t sc_full[2];
   uint64_t sc_empty[2];
   uint64_t acc_full[2];
@@ -122,7 +129,7 @@ __device__ __forceinline__ TileInfo decode_tile(const Bars& b, int E, int NT, in
 __device__ __forceinline__ float silu_clamped(float hg, float hu) {
   const float g = fminf(hg, 7.f);
   const float u = fminf(fmaxf(hu, -7.f), 7.f);
-  return (u + 1.f) * g * (1.f / (1.f + __expf(-1.702f * g)));
+  return (u + 1.f) * g * __frcp_rn(1.f + __expf(-1.702f * g));
 }
 
 template <bool kGateUp>
@@ -148,8 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&b.full_ab[s], 1);
-      mbar_init(&b.full_b[s], kDeqWarps);
       mbar_init(&b.empty[s], 1);
+    }
+    for (int s = 0; s < kTStages; ++s) {
+      mbar_init(&b.full_b[s], kDeqWarps);
+      mbar_init(&b.tfree[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&b.sc_full[i], 1);
@@ -195,7 +205,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           mbar_arrive_expect_tx(&b.full_ab[s], kTokBytes + kPackBytes);
           tma_load_2d(smem + kOffTok + s * kTokBytes, &mapA, &b.full_ab[s], kt * kBK, ti.row0);
+          // the 32 packed bytes of a row per K step land as two 16-byte halves, [half][row][16 B], so
+          // that the dequant warps' 16-byte reads of consecutive rows are contiguous
           tma_load_2d(smem + kOffPack + s * kPackBytes, &mapP, &b.full_ab[s], kt * (kBK / 2), prow);
+          tma_load_2d(smem + kOffPack + s * kPackBytes + kPackBytes / 2, &mapP, &b.full_ab[s], kt * (kBK / 2) + 16,
+                      prow);
         }
       }
       // Drain: wait (bounded) for copies still in flight before the CTA may exit.
@@ -213,7 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sub = warp & 3, h = (warp - kDeqWarp0) >> 2;
     const int r = sub * 32 + lane;
     const uint32_t t_lane = tmem_base + ((uint32_t)(sub * 32) << 16) + kAColBase + h * kDeqCols;
-    const int pk_off = r * 32 + h * kDeqCols;        // byte offset of this thread's packed bytes
+    // byte offset of this thread's packed bytes: half (h * kDeqCols) / 16, row r, then the rest of the offset
+    const int pk_off = ((h * kDeqCols) / 16) * (kPackBytes / 2) + r * 16 + (h * kDeqCols) % 16;
     const int sc_blk = (h * kDeqCols) / 16;          // MX block of the step (0 or 1)
     int it = 0, tc = 0;
     bool ok = true;
@@ -222,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait_bar(&b.sc_full[sb], (tc >> 1) & 1, lim, abort_flag, a.status);
       if (!ok) break;
       const uint8_t* sc = smem + kOffSc + sb * scbytes + r * KB + sc_blk;
-      uint32_t va[kDeqCols], vb[kDeqCols];  // step k in va (being stored), step k+1 converted into vb
+      uint32_t va[kDeqCols];  // the converted step
       auto convert = [&](int kt, int s, uint32_t* v) {
         const uint32_t sv = sc[kt * 2];
         const uint8_t* src = smem + kOffPack + s * kPackBytes + pk_off;
@@ -243,22 +258,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       convert(0, it % kStages, va);
       for (int kt = 0; kt < KT; ++kt, ++it) {
-        const int s = it % kStages;
-        if constexpr (kDeqCols == 16) tmem_st16(t_lane + s * kAStageCols, va);
-        else tmem_st8(t_lane + s * kAStageCols, va);
-        const bool more = kt + 1 < KT;
-        if (more) {  // convert the next step while this store drains
-          ok = wait_bar(&b.full_ab[(it + 1) % kStages], ((it + 1) / kStages) & 1, lim, abort_flag, a.status);
-          if (ok) convert(kt + 1, (it + 1) % kStages, vb);
+        // Step it goes to TMEM stage it % kTStages once the MMAs of step it - kTStages are done; the
+        // stage is handed to the MMA warp as soon as it is written, then the next step is converted
+        // (its shared-memory stage usually landed long before: the TMA ring is deeper than this one).
+        const int st = it % kTStages;
+        if (it >= kTStages) {
+          ok = wait_bar(&b.tfree[st], ((it / kTStages) - 1) & 1, lim, abort_flag, a.status);
+          if (!ok) break;
+          tc_fence_after();
         }
+        if constexpr (kDeqCols == 16) tmem_st16(t_lane + st * kAStageCols, va);
+        else tmem_st8(t_lane + st * kAStageCols, va);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&b.full_b[s]);
-        if (!ok) break;
-        if (more) {
-#pragma unroll
-          for (int i = 0; i < kDeqCols; ++i) va[i] = vb[i];
+        if (lane == 0) mbar_arrive(&b.full_b[st]);
+        if (kt + 1 < KT) {
+          ok = wait_bar(&b.full_ab[(it + 1) % kStages], ((it + 1) / kStages) & 1, lim, abort_flag, a.status);
+          if (!ok) break;
+          convert(kt + 1, (it + 1) % kStages, va);
         }
       }
       if (!ok) break;
@@ -277,18 +295,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * kAccCols;
         for (int kt = 0; kt < KT; ++kt, ++it) {
-          const int s = it % kStages;
-          const uint32_t par = (it / kStages) & 1;
-          ok = wait_bar(&b.full_ab[s], par, lim, abort_flag, a.status) &&
-               wait_bar(&b.full_b[s], par, lim, abort_flag, a.status);
+          const int s = it % kStages, st = it % kTStages;
+          ok = wait_bar(&b.full_ab[s], (it / kStages) & 1, lim, abort_flag, a.status) &&
+               wait_bar(&b.full_b[st], (it / kTStages) & 1, lim, abort_flag, a.status);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + kAColBase + s * kAStageCols;
+          const uint32_t a_tmem = tmem_base + kAColBase + st * kAStageCols;
           const uint32_t sbb = smem_u32(smem + kOffTok + s * kTokBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             umma_bf16_ts(d_tmem, a_tmem + kk * 8, smem_desc_k128(sbb + kk * 32), idesc, (kt | kk) ? 1u : 0u);
           umma_commit(&b.empty[s]);
+          umma_commit(&b.tfree[st]);
         }
         if (!ok) break;
         umma_commit(&b.acc_full[ab]);
@@ -330,12 +348,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(tbase + c0, r);
         tmem_wait_ld();
         if (kGateUp) {
-          // even lanes: gate row n with the up row n+1 of the odd neighbour -> act[token][n/2]
+          // Lane pair (2i, 2i+1) holds gate row 2i and up row 2i+1 of columns j: for each pair of
+          // columns (j, j+1) the even lane computes act of column j and the odd lane of column j+1,
+          // one exchange per pair, no idle lanes -> act[token][row / 2].
+          const bool odd = lane & 1;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float v = __uint_as_float(r[j]) + bias;
-            const float u = __shfl_xor_sync(0xffffffffu, v, 1);
-            if ((lane & 1) == 0) ep.act[warp][j][lane >> 1] = (uint16_t)float_to_bf16_bits(silu_clamped(v, u));
+          for (int j = 0; j < 16; j += 2) {
+            const float v0 = __uint_as_float(r[j]) + bias, v1 = __uint_as_float(r[j + 1]) + bias;
+            const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
+            const float g = odd ? recv : v0;  // gate of the column this lane computes
+            const float u = odd ? v1 : recv;  // up of that column
+            ep.act[warp][j + (odd ? 1 : 0)][lane >> 1] = (uint16_t)float_to_bf16_bits(silu_clamped(g, u));
           }
           __syncwarp();
           // lane L stores 8 outputs (16 bytes) of token c0 + L/2
@@ -379,7 +402,7 @@ cudaError_t launch(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStrea
   if (!make_map_2d(&mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_ptr, a.K, a.total_rows, kBK, kTN,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (!make_map_2d(&mapP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.blocks, a.K / 2, (uint64_t)a.E * a.N, kBK / 2, kWM,
+  if (!make_map_2d(&mapP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.blocks, a.K / 2, (uint64_t)a.E * a.N, 16, kWM,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const size_t smem = smem_total(a.K);

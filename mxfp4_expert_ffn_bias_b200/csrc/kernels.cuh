@@ -34,6 +34,9 @@ __global__ void route_small_kernel(const uint16_t* __restrict__ x, const float* 
                                    const float* __restrict__ rb, int T, int H, int E, int k, int HC,
                                    float* __restrict__ partial, float* __restrict__ pmax,
                                    float* __restrict__ logits, int* __restrict__ ticket, RouteOut o);
+size_t route_cluster_smem_bytes(int T, int H, int E, int k, int CS);
+__global__ void route_cluster_kernel(const uint16_t* __restrict__ x, const float* __restrict__ rw,
+                                     const float* __restrict__ rb, int T, int H, int E, int k, RouteOut o);
 constexpr int kRouteTickets = 1 + 32;  // small-T router: final ticket + one per group of 8 experts (E <= 256)
 __global__ void split_router_kernel(const float* __restrict__ rw, size_t n, uint16_t* __restrict__ w3);
 __global__ void route_mma_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w3,

@@ -389,6 +389,235 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int* __restric
   }
 }
 
+// L2 prefetch of [p, p + bytes) widened to 16-byte boundaries (the range must lie inside an allocation
+// whose ends are 16-byte aligned). Issued before the grid dependency wait: a prefetch only warms L2,
+// which stays coherent with any write the previous kernel still makes.
+__device__ __forceinline__ void prefetch_range(const void* p, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p) & ~uintptr_t(15);
+  const uintptr_t b = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t(15);
+  if (b > a) bulk_prefetch_l2(reinterpret_cast<const void*>(a), (uint32_t)(b - a));
+}
+
+// ---------------------------------------------------------------- small-T router on one thread-block cluster
+
+// For T <= kSmallT: one cluster of CS CTAs. CTA c stages hidden columns
+// [c*HS, (c+1)*HS) of x (fp32) and of the router weight (transposed) in its
+// shared memory and computes the partial logits of every (token, expert) over
+// them with fp32 FMAs, plus each token's partial max|x|. After a cluster
+// barrier, token t is finished by CTA t % CS: its logits are the partial sums
+// read from the CTAs' shared memory in CTA order (distributed shared memory)
+// plus the bias; top-k, softmax and c_t follow, and the selected experts are
+// written into CTA 0's shared memory. After a second barrier CTA 0 runs the
+// stable counting sort of all pairs. No global round trip inside the router.
+struct ClusterLayout {
+  int HS, Tp, Ep;
+  size_t xT, wT, part, amax, sel, cnt, total;
+};
+
+__host__ __device__ inline ClusterLayout cluster_layout(int T, int H, int E, int k, int CS) {
+  ClusterLayout L;
+  L.HS = H / CS;
+  L.Tp = (T + 3) & ~3;
+  L.Ep = (E + 3) & ~3;
+  L.xT = 0;
+  L.wT = L.xT + (size_t)L.HS * L.Tp * 4;
+  L.part = L.wT + (size_t)L.HS * L.Ep * 4;
+  L.amax = L.part + (size_t)T * E * 4;
+  L.sel = L.amax + (size_t)L.Tp * 4;
+  L.cnt = L.sel + (size_t)T * k * 4;
+  L.total = L.cnt + (size_t)3 * 260 * 4;
+  return L;
+}
+
+size_t route_cluster_smem_bytes(int T, int H, int E, int k, int CS) { return cluster_layout(T, H, E, k, CS).total; }
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_to_cta(const void* p, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(cta));
+  return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__global__ void __launch_bounds__(512, 1) route_cluster_kernel(const uint16_t* __restrict__ x,
+                                                               const float* __restrict__ rw,
+                                                               const float* __restrict__ rb, int T, int H, int E,
+                                                               int k, RouteOut o) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int CS = (int)gridDim.x;  // one cluster spans the grid
+  const uint32_t rank = cluster_ctarank();
+  {
+    const int hs = H / CS, hb = (int)rank * hs;
+    if ((int)threadIdx.x < T) prefetch_range(x + (size_t)threadIdx.x * H + hb, (size_t)hs * 2);
+    else if ((int)threadIdx.x >= 64 && (int)threadIdx.x - 64 < E)
+      prefetch_range(rw + (size_t)(threadIdx.x - 64) * H + hb, (size_t)hs * 4);
+  }
+  pdl_wait_and_trigger();
+  const ClusterLayout L = cluster_layout(T, H, E, k, CS);
+  float* xT = reinterpret_cast<float*>(sm + L.xT);    // [HS][Tp]
+  float* wT = reinterpret_cast<float*>(sm + L.wT);    // [HS][Ep]
+  float* part = reinterpret_cast<float*>(sm + L.part);  // [T][E]
+  float* amax = reinterpret_cast<float*>(sm + L.amax);  // [Tp]
+  int* s_sel = reinterpret_cast<int*>(sm + L.sel);    // [T*k] (CTA 0)
+  int* s_cnt = reinterpret_cast<int*>(sm + L.cnt);
+  int* s_off = s_cnt + 260;
+  int* s_mt = s_off + 260;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nthr = blockDim.x;
+  const int HS = L.HS, Tp = L.Tp, Ep = L.Ep;
+  const int h0 = (int)rank * HS;
+
+  // stage this CTA's columns (unrolled so that several loads are in flight)
+#pragma unroll 4
+  for (int i = tid; i < Tp * (HS / 2); i += nthr) {
+    const int t = i / (HS / 2), c2 = i - t * (HS / 2);
+    uint32_t v = 0;
+    if (t < T) v = *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + 2 * c2);
+    xT[(2 * c2) * Tp + t] = bf16_bits_to_float(v & 0xFFFF);
+    xT[(2 * c2 + 1) * Tp + t] = bf16_bits_to_float(v >> 16);
+  }
+#pragma unroll 4
+  for (int i = tid; i < Ep * (HS / 4); i += nthr) {
+    const int e = i / (HS / 4), c4 = i - e * (HS / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e < E) v = *reinterpret_cast<const float4*>(rw + (size_t)e * H + h0 + 4 * c4);
+    wT[(4 * c4) * Ep + e] = v.x;
+    wT[(4 * c4 + 1) * Ep + e] = v.y;
+    wT[(4 * c4 + 2) * Ep + e] = v.z;
+    wT[(4 * c4 + 3) * Ep + e] = v.w;
+  }
+  __syncthreads();
+  // partial max|x| per token over this CTA's columns
+  for (int t = warp; t < Tp; t += nthr / 32) {
+    float m = 0.f;
+    for (int c = lane; c < HS; c += 32) m = fmaxf(m, fabsf(xT[c * Tp + t]));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) amax[t] = m;
+  }
+  // partial logits: 4 tokens x 4 experts per thread, `ks` adjacent lanes split the columns
+  const int nT4 = Tp / 4, nE4 = Ep / 4, ntiles = nT4 * nE4;
+  int ks = 1;
+  while (ks < 32 && ntiles * ks * 2 <= nthr) ks *= 2;
+  const int kp = tid % ks;
+  const int per_round = nthr / ks;
+  const int rounds = (ntiles + per_round - 1) / per_round;
+  for (int rd = 0; rd < rounds; ++rd) {  // same trip count for every thread: the shuffles below are uniform
+    const int tile = rd * per_round + tid / ks;
+    const bool act = tile < ntiles;
+    const int t4 = act ? tile / nE4 : 0, e4 = act ? tile - t4 * nE4 : 0;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    if (act) {
+      for (int c = kp; c < HS; c += ks) {
+        const float4 xv = *reinterpret_cast<const float4*>(xT + c * Tp + 4 * t4);
+        const float4 wv = *reinterpret_cast<const float4*>(wT + c * Ep + 4 * e4);
+        const float xa[4] = {xv.x, xv.y, xv.z, xv.w}, wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], wa[j], acc[i][j]);
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1)
+      if (off < ks)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], off);
+    if (act && kp == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int t = 4 * t4 + i, e = 4 * e4 + j;
+          if (t < T && e < E) part[t * E + e] = acc[i][j];
+        }
+    }
+  }
+  cluster_sync_all();  // every CTA's partial logits and max|x| are in place
+
+  // tokens t = rank, rank + CS, ...: one warp each
+  const int EJ = (E + 31) / 32;
+  for (int t = (int)rank + CS * warp; t < T; t += CS * (nthr / 32)) {
+    float lg[kMaxEJ];
+#pragma unroll
+    for (int j = 0; j < kMaxEJ; ++j) {
+      const int e = lane + 32 * j;
+      float v = -INFINITY;
+      if (j < EJ && e < E) {
+        v = 0.f;
+        for (int c = 0; c < CS; ++c) v += ld_cluster_f32(map_to_cta(part + t * E + e, (uint32_t)c));
+        v += rb[e];
+      }
+      lg[j] = v;
+    }
+    int sele[8];
+    float selv[8], w[8];
+    warp_topk(lg, EJ, E, k, sele, selv);
+    float m = 0.f;
+    for (int c = lane; c < CS; c += 32) m = fmaxf(m, ld_cluster_f32(map_to_cta(amax + t, (uint32_t)c)));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) {
+      softmax_k(selv, k, w);
+      o.xexp[t] = token_exponent(m);
+      for (int s = 0; s < k; ++s) {
+        o.idx[t * k + s] = sele[s];
+        o.w[t * k + s] = w[s];
+        st_cluster_u32(map_to_cta(s_sel + t * k + s, 0u), (uint32_t)sele[s]);
+      }
+    }
+  }
+  cluster_sync_all();  // all selections are in CTA 0; no CTA reads another's memory after this
+  if (rank != 0) return;
+
+  // CTA 0: stable counting sort of the T*k pairs by expert
+  const int Tk = T * k;
+  for (int e = tid; e < E; e += nthr) {
+    int c = 0;
+    for (int p = 0; p < Tk; ++p) c += (s_sel[p] == e);
+    s_cnt[e] = c;
+    o.counts[e] = c;
+  }
+  __syncthreads();
+  prefix_counts(s_cnt, E, s_off, s_mt);
+  __syncthreads();
+  for (int i = tid; i <= E; i += nthr) {
+    o.offsets[i] = s_off[i];
+    o.mt_off[i] = s_mt[i];
+  }
+  if (tid == 0) {
+    int n = 0;
+    for (int j = 0; j < E; ++j)
+      if (s_cnt[j] > 0) o.touched[n++] = j;
+    *o.n_touched = n;
+  }
+  for (int p = tid; p < Tk; p += nthr) {
+    const int e = s_sel[p];
+    int rank_e = 0;
+    for (int j = 0; j < p; ++j) rank_e += (s_sel[j] == e);
+    o.perm[s_off[e] + rank_e] = p;
+  }
+}
+
 // ---------------------------------------------------------------- small-T router (one launch)
 
 // For T <= kSmallT, in three phases inside one launch:
@@ -413,10 +642,13 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
                                                           int HC, float* __restrict__ partial,
                                                           float* __restrict__ pmax, float* __restrict__ logits,
                                                           int* __restrict__ ticket, RouteOut o) {
-  pdl_wait_and_trigger();
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
   const int eg = blockIdx.x, hc = blockIdx.y, nHC = gridDim.y, nEG = gridDim.x;
+  if ((int)threadIdx.x < T) prefetch_range(x + (size_t)threadIdx.x * H + hc * HC, (size_t)HC * 2);
+  else if (threadIdx.x >= 64 && threadIdx.x < 72 && eg * 8 + (int)threadIdx.x - 64 < E)
+    prefetch_range(rw + (size_t)(eg * 8 + threadIdx.x - 64) * H + hc * HC, (size_t)HC * 4);
+  pdl_wait_and_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h0 = hc * HC;
   const int XS = HC + 2, WS = HC + 1;
