@@ -84,6 +84,21 @@ def gateup_units(cfg, n_touched: int, T: int):
     return bytes_alg, flops
 
 
+# ---------------------------------------------------------------- multi-rank bookkeeping
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value of x over all ranks (every rank gets it): the job's time is its slowest rank's."""
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank runs its own replica on its own batch (weak scaling)."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- DRAM traffic of the roofline kernels
 
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the benchmark's own
@@ -345,11 +360,9 @@ def run_ours(args):
         dist.barrier()
     total_ms = sum(r["step_ms"])
     if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = max_over_ranks(total_ms, dist, "cuda")
     ms_step = total_ms / args.steps
-    value = world * T / (ms_step / 1e3)
+    value = job_value(world, T, ms_step)
 
     bytes_alg, flops_alg = layer_units(cfg, r["n_touched"], T)
     gu_bytes, gu_flops = gateup_units(cfg, r["n_touched"], T)

@@ -165,8 +165,14 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
 // Both MMAs of a block cover exactly its 32 elements, so the fp32 result is
 // scaled by the row's 2^(s-127) and added to the accumulator.
 
-constexpr int kMmaUnroll = 8;  // MX blocks per pipeline group (two groups in flight)
-constexpr int kMmaWarps = 6;   // warps per block (measured best of 4, 6, 8 on the gpt-oss decode shapes)
+#ifndef MOE_GEMV_UNROLL
+#define MOE_GEMV_UNROLL 8
+#endif
+constexpr int kMmaUnroll = MOE_GEMV_UNROLL;  // MX blocks per pipeline group (two groups in flight)
+#ifndef MOE_GEMV_WARPS
+#define MOE_GEMV_WARPS 6
+#endif
+constexpr int kMmaWarps = MOE_GEMV_WARPS;    // warps per block (measured best of 4, 6, 8 on the gpt-oss decode shapes)
 constexpr int kMmaRows = 16 * kMmaWarps;  // weight rows per block
 
 __device__ __forceinline__ uint32_t ldg_u32(const void* p) {

@@ -1,0 +1,74 @@
+"""Host-side logic of bench.py that needs no GPU: the max-over-ranks reduction on two gloo ranks,
+the whole-job throughput, the algorithmic units, and the reference arm launched on two ranks."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from gen.synth import CONFIGS  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out[rank] = bench.max_over_ranks(1.5 + 2.0 * rank, dist, "cpu")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_on_two_gloo_ranks():
+    port = _free_port()
+    out = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_rank_main, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+    assert dict(out) == {0: 3.5, 1: 3.5}
+
+
+def test_job_value_is_the_sum_of_replicas():
+    assert bench.job_value(1, 8, 0.1) == pytest.approx(80000.0)
+    assert bench.job_value(4, 8, 0.1) == pytest.approx(4 * 80000.0)
+
+
+def test_layer_units_of_the_tiny_layer():
+    cfg = CONFIGS["tiny"]
+    b, f = bench.layer_units(cfg, n_touched=5, T=cfg.T)
+    per_expert = 2 * cfg.I * (cfg.H // 2 + cfg.H // 32) + cfg.H * (cfg.I // 2 + cfg.I // 32) + 2 * (2 * cfg.I + cfg.H)
+    assert b == 5 * per_expert + cfg.E * cfg.H * 4 + cfg.E * 4 + 2 * cfg.T * cfg.H * 2
+    assert f == 2 * cfg.T * cfg.k * 3 * cfg.I * cfg.H + 2 * cfg.T * cfg.E * cfg.H
+
+
+def test_launches_per_call():
+    assert bench.launches_per_call(8, decode=True) == 4
+    assert bench.launches_per_call(4096, decode=False) == 7
+
+
+def test_reference_arm_on_two_ranks_prints_one_line():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0", "--config", "tiny"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
