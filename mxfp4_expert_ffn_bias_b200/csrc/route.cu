@@ -480,10 +480,11 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(const uint16_t* _
   const int HS = L.HS, Tp = L.Tp, Ep = L.Ep;
   const int h0 = (int)rank * HS;
 
-  // stage this CTA's columns (unrolled so that several loads are in flight)
+  // stage this CTA's columns, transposed; consecutive threads take consecutive tokens / experts so that
+  // the shared-memory stores are conflict-free (unrolled so that several loads are in flight)
 #pragma unroll 4
   for (int i = tid; i < Tp * (HS / 2); i += nthr) {
-    const int t = i / (HS / 2), c2 = i - t * (HS / 2);
+    const int c2 = i / Tp, t = i - c2 * Tp;
     uint32_t v = 0;
     if (t < T) v = *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + 2 * c2);
     xT[(2 * c2) * Tp + t] = bf16_bits_to_float(v & 0xFFFF);
@@ -491,7 +492,7 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(const uint16_t* _
   }
 #pragma unroll 4
   for (int i = tid; i < Ep * (HS / 4); i += nthr) {
-    const int e = i / (HS / 4), c4 = i - e * (HS / 4);
+    const int c4 = i / Ep, e = i - c4 * Ep;
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (e < E) v = *reinterpret_cast<const float4*>(rw + (size_t)e * H + h0 + 4 * c4);
     wT[(4 * c4) * Ep + e] = v.x;
@@ -563,8 +564,13 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(const uint16_t* _
       const int e = lane + 32 * j;
       float v = -INFINITY;
       if (j < EJ && e < E) {
+        float pc[16];  // the CTAs' partial sums, loaded together, added in CTA order
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pc[c] = c < CS ? ld_cluster_f32(map_to_cta(part + t * E + e, (uint32_t)c)) : 0.f;
         v = 0.f;
-        for (int c = 0; c < CS; ++c) v += ld_cluster_f32(map_to_cta(part + t * E + e, (uint32_t)c));
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if (c < CS) v += pc[c];
         v += rb[e];
       }
       lg[j] = v;
