@@ -104,7 +104,16 @@ def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from one ncu capture of the benchmark's own
 # workload (profiles/ holds the summaries and the commands). A value is reported only while the
 # sources of the kernel's translation unit hash to what they were when it was captured.
-TRAFFIC = {}
+_GEMV_TU = ["mxfp4_expert_ffn_bias_b200/csrc/gemv.cu", "mxfp4_expert_ffn_bias_b200/csrc/common.cuh",
+            "mxfp4_expert_ffn_bias_b200/csrc/kernels.cuh", "mxfp4_expert_ffn_bias_b200/csrc/mx_dequant.cuh",
+            "include/moe.h"]
+_GEMM_TU = ["mxfp4_expert_ffn_bias_b200/csrc/gemm_sm100.cu"] + _GEMV_TU[1:]
+TRAFFIC = {
+    # profiles/decode-kernels_gpt-oss-20b-decode.md: 194.23 MB read + 3.89 MB written
+    ("moe::gemv_mma_kernel<true>", "gpt-oss-20b-decode"): {"bytes": 198121728, "files": _GEMV_TU, "hash": "a7f9a061aa33c431"},
+    # profiles/prefill-kernels_gpt-oss-20b-prefill.md: 377.50 MB read + 82.16 MB written
+    ("moe::grouped_mxfp4_gemm<true>", "gpt-oss-20b-prefill"): {"bytes": 459654144, "files": _GEMM_TU, "hash": "af2cbb84f3ab64b7"},
+}
 
 
 def _tu_hash(files):
