@@ -109,11 +109,14 @@ moe_status_t moe_forward(moe_handle_t h, const void* x, const float* router_w, c
                          void* out, void* stream);
 
 /*
- * Same as moe_forward, but x and out are HOST pointers (bf16 [T, H] each;
- * pinned memory gives the best copy speed). The call copies x to the
- * handle's device staging buffer, runs the layer, copies the result back
- * and synchronises `stream` before returning, so out is valid on return.
- * The weight arguments are device pointers as in moe_forward.
+ * Same as moe_forward, but x and out are HOST pointers (bf16 [T, H] each).
+ * Page-locked memory that is mapped into the device address space (e.g.
+ * cudaHostAlloc on a unified-addressing system), 16-byte aligned, is accessed
+ * by the kernels directly: a copy kernel moves x into the handle's device
+ * staging buffer and the last kernel writes out in place. Other host memory
+ * goes through cudaMemcpyAsync both ways. The call synchronises `stream`
+ * before returning, so out is valid on return. The weight arguments are
+ * device pointers as in moe_forward.
  */
 moe_status_t moe_forward_hostio(moe_handle_t h, const void* x_host, const float* router_w, const float* router_b,
                                 const uint8_t* gate_up_blocks, const uint8_t* gate_up_scales,

@@ -52,6 +52,7 @@ __global__ void route_scatter_kernel(const int* __restrict__ idx, const int* __r
                                      int* __restrict__ perm, uint16_t* __restrict__ x_perm);
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int* __restrict__ perm, int k, int H,
                                    uint16_t* __restrict__ x_perm);
+__global__ void copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n);
 __global__ void combine_kernel(const float* __restrict__ slot, int T, int H, int k, uint16_t* __restrict__ out);
 __global__ void debug_dequant_kernel(const uint8_t* __restrict__ blocks, const uint8_t* __restrict__ scales,
                                      int rows, int cols, uint16_t* __restrict__ out);

@@ -291,6 +291,17 @@ moe_status_t enqueue_route(moe_handle_t h, const void* x, const float* rw, const
   return MOE_OK;
 }
 
+// Device address of a host buffer the GPU can access directly (page-locked and mapped), else null.
+void* mapped_device_ptr(const void* host) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, host) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (at.type != cudaMemoryTypeHost || !at.devicePointer) return nullptr;
+  return at.devicePointer;
+}
+
 bool use_decode(const moe_ctx* h, int T) {
   if (h->path_opt == 1) return true;
   if (h->path_opt == 2) return false;
@@ -424,11 +435,23 @@ MOE_API moe_status_t moe_forward_hostio(moe_handle_t h, const void* x_host, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   h->last_stream = st;
   const size_t bytes = (size_t)T * h->H * sizeof(uint16_t);
-  MOE_CHECK_CUDA(cudaMemcpyAsync(h->ws.x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
+  // Page-locked host buffers mapped into the device address space are read and written by the kernels
+  // directly (no copy-engine round trips for small batches); other host memory goes through copies.
+  const void* dx = mapped_device_ptr(x_host);
+  void* dout = mapped_device_ptr(out_host);
+  if (dx && (reinterpret_cast<uintptr_t>(dx) & 15u) == 0) {
+    const size_t n16 = bytes / 16;
+    const int blocks = (int)((n16 + 255) / 256 < 1184 ? (n16 + 255) / 256 : 1184);
+    MOE_CHECK_CUDA(launch_pdl(copy16_kernel, dim3(blocks), dim3(256), 0, st, static_cast<const uint4*>(dx),
+                              reinterpret_cast<uint4*>(h->ws.x_stage), n16));
+  } else {
+    MOE_CHECK_CUDA(cudaMemcpyAsync(h->ws.x_stage, x_host, bytes, cudaMemcpyHostToDevice, st));
+  }
+  const bool direct_out = dout && (reinterpret_cast<uintptr_t>(dout) & 15u) == 0;
   s = enqueue_forward(h, h->ws.x_stage, router_w, router_b, gate_up_blocks, gate_up_scales, gate_up_bias,
-                      down_blocks, down_scales, down_bias, T, h->ws.out_stage, st);
+                      down_blocks, down_scales, down_bias, T, direct_out ? dout : h->ws.out_stage, st);
   if (s != MOE_OK) return s;
-  MOE_CHECK_CUDA(cudaMemcpyAsync(out_host, h->ws.out_stage, bytes, cudaMemcpyDeviceToHost, st));
+  if (!direct_out) MOE_CHECK_CUDA(cudaMemcpyAsync(out_host, h->ws.out_stage, bytes, cudaMemcpyDeviceToHost, st));
   MOE_CHECK_CUDA(cudaStreamSynchronize(st));
   return MOE_OK;
 }

@@ -806,6 +806,14 @@ __global__ void __launch_bounds__(128) gather_rows_kernel(const uint16_t* __rest
 }
 
 // out[t, j] = bf16( sum_{s=0..k-1} slot[t*k+s, j] ), summed in slot order.
+// Copy of n 16-byte units (host-io: token rows from page-locked, device-mapped host memory into the
+// workspace, so that the layer's many readers of x read device memory).
+__global__ void __launch_bounds__(256) copy16_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n) {
+  pdl_wait_and_trigger();
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ slot, int T, int H, int k,
                                                       uint16_t* __restrict__ out) {
   pdl_wait_and_trigger();

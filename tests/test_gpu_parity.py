@@ -242,23 +242,30 @@ def test_decode_and_prefill_paths_agree(moe):
     assert s["max_err"] <= 2e-2 * s["max_ref"] + 1e-3
 
 
-def test_hostio_matches_device_path(moe):
-    cfg = CONFIGS["tiny"]
-    inp = inputs_for("tiny")
+@pytest.mark.parametrize("name", ["tiny", "gpt-oss-20b-decode"])
+@pytest.mark.parametrize("pinned", [True, False])
+def test_hostio_matches_device_path(moe, name, pinned):
+    """Host buffers: page-locked (read and written by the kernels in place) or pageable (copied)."""
+    cfg = CONFIGS[name]
+    inp = inputs_for(name)
     dev = to_device(inp)
     T = cfg.T
     h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
     try:
         out_dev = run_forward(moe, h, dev, T, cfg.H)
         torch.cuda.synchronize()
-        x_host = torch.from_numpy(inp["x"].view(np.int16).copy()).pin_memory()
-        out_host = torch.empty((T, cfg.H), dtype=torch.int16).pin_memory()
-        moe.moe_forward_hostio(h, x_host, dev["router_w"], dev["router_b"], dev["gate_up_blocks"],
-                               dev["gate_up_scales"], dev["gate_up_bias"], dev["down_blocks"], dev["down_scales"],
-                               dev["down_bias"], T, out_host)
+        x_host = torch.from_numpy(inp["x"].view(np.int16).copy())
+        out_host = torch.empty((T, cfg.H), dtype=torch.int16)
+        if pinned:
+            x_host, out_host = x_host.pin_memory(), out_host.pin_memory()
+        for _ in range(2):
+            out_host.zero_()
+            moe.moe_forward_hostio(h, x_host, dev["router_w"], dev["router_b"], dev["gate_up_blocks"],
+                                   dev["gate_up_scales"], dev["gate_up_bias"], dev["down_blocks"],
+                                   dev["down_scales"], dev["down_bias"], T, out_host)
+            assert np.array_equal(out_host.numpy(), out_dev.view(torch.int16).cpu().numpy())
     finally:
         moe.moe_destroy(h)
-    assert np.array_equal(out_host.numpy(), out_dev.view(torch.int16).cpu().numpy())
 
 
 def test_invalid_token_counts_rejected(moe):
