@@ -109,6 +109,22 @@ inline EncodeTiledFn get_encode() {
   return fn;
 }
 
+// 3-D view of a row-major matrix [rows][row_bytes]: element (x, y, z) at y * row_bytes + (z * chunk + x) * esize,
+// i.e. the columns of each row cut into chunks of `chunk` elements; a box takes box_z consecutive chunks of
+// box_y rows, landing as [z][y][x]. Out-of-range elements read as zero.
+inline bool make_map_3d_chunks(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t chunk,
+                               uint64_t rows, uint64_t nchunks, uint64_t row_bytes, uint32_t box_y, uint32_t box_z,
+                               CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {chunk, rows, nchunks};
+  cuuint64_t strides[2] = {row_bytes, chunk * (uint64_t)esize};
+  cuuint32_t box[3] = {(cuuint32_t)chunk, box_y, box_z};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Row-major 2-D tensor [outer][inner] of `esize`-byte elements; box of
 // box_outer rows x box_inner elements; out-of-range elements read as zero.
 inline bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr, uint64_t inner,
@@ -223,6 +239,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// 3-D tiled TMA load into shared memory, completion counted on `bar` (bytes).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 

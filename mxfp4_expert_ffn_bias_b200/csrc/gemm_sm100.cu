@@ -50,10 +50,7 @@ namespace {
 
 constexpr int kWM = 128;                    // weight rows per tile (MMA M, TMEM lanes)
 constexpr int kTN = kBM;                    // token rows per tile (MMA N)
-#ifndef MOE_GEMM_STAGES
-#define MOE_GEMM_STAGES 6
-#endif
-constexpr int kStages = MOE_GEMM_STAGES;    // TMA ring (token + packed tiles) in shared memory
+constexpr int kStages = 3;                  // TMA ring in shared memory; one stage = two K steps
 constexpr int kTStages = 4;                 // TMEM ring of dequantised A stages
 #ifndef MOE_DEQ_WARPS
 #define MOE_DEQ_WARPS 8  // measured: 8 (900 us) beat 16 (972 us) on the 20b prefill gate_up
@@ -71,11 +68,13 @@ constexpr int kTmemCols = 512;
 static_assert(kAColBase + kTStages * kAStageCols <= kTmemCols, "TMEM budget");
 constexpr int kMaxE = 256;
 
-constexpr int kTokBytes = kTN * 128;        // one token stage (64 bf16 per row)
-constexpr int kPackBytes = kWM * 32;        // one packed weight stage: two halves [2][kWM rows][16 bytes]
+constexpr int kTokBytes = kTN * 128;        // tokens of one K step (64 bf16 per row, 128B swizzle)
+constexpr int kPackBytes = kWM * 32;        // packed weights of one K step: [2 halves][kWM rows][16 bytes]
+constexpr int kTokStage = 2 * kTokBytes;    // one ring stage: two K steps of tokens ...
+constexpr int kPackStage = 2 * kPackBytes;  // ... and of packed weights, each landed by ONE 3-D TMA copy
 constexpr int kOffTok = 0;
-constexpr int kOffPack = kOffTok + kStages * kTokBytes;
-constexpr int kOffEpi = kOffPack + kStages * kPackBytes;  // epilogue staging (see Epi)
+constexpr int kOffPack = kOffTok + kStages * kTokStage;
+constexpr int kOffEpi = kOffPack + kStages * kPackStage;  // epilogue staging (see Epi)
 struct Epi {
   uint16_t act[4][16][16];  // per epilogue warp: 16 tokens x 16 SwiGLU outputs (bf16), transposed for stores
   int pair[2][kBM];         // per accumulator buffer: (token, slot) pair of each token row of the tile
@@ -84,8 +83,8 @@ struct Epi {
 constexpr int kOffSc = kOffEpi + (int)((sizeof(Epi) + 127) / 128 * 128);  // 2 scale buffers of kWM * KB bytes
 
 struct __align__(8) Bars {
-  uint64_t full_ab[kStages];   // TMA landed (token + packed tiles)
-  uint64_t empty[kStages];     // MMAs of the step done (shared-memory stage free)
+  uint64_t full_ab[kStages];   // TMA landed (token + packed tiles of two K steps)
+  uint64_t empty[kStages];     // MMAs of the stage's K steps done (shared-memory stage free)
   uint64_t full_b[kTStages];   // TMEM A stage written by the dequant warps
   uint64_t tfree[kTStages];    // MMAs that read the TMEM A stage done
   uint64_t sc_full[2];
@@ -140,7 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int KB = a.K / 32;
-  const int KT = a.K / kBK;
+  const int KT = a.K / kBK;      // K steps of a tile
+  const int SS = (KT + 1) / 2;   // ring stages of a tile (two K steps each)
   const int NT = (a.N + kWM - 1) / kWM;
   const int scbytes = kWM * KB;
   Bars& b = *reinterpret_cast<Bars*>(smem + kOffSc + 2 * scbytes);
@@ -199,17 +199,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(smem + kOffSc + sb * scbytes, a.scales + ((size_t)ti.e * a.N + n0) * KB, wrows * KB,
                   &b.sc_full[sb]);
         const int prow = ti.e * a.N + n0;
-        for (int kt = 0; kt < KT; ++kt, ++it) {
+        for (int j = 0; j < SS; ++j, ++it) {  // it: ring stages issued, two K steps each
           const int s = it % kStages;
           ok = wait_bar(&b.empty[s], ((it / kStages) & 1) ^ 1, lim, abort_flag, a.status);
           if (!ok) break;
-          mbar_arrive_expect_tx(&b.full_ab[s], kTokBytes + kPackBytes);
-          tma_load_2d(smem + kOffTok + s * kTokBytes, &mapA, &b.full_ab[s], kt * kBK, ti.row0);
-          // the 32 packed bytes of a row per K step land as two 16-byte halves, [half][row][16 B], so
-          // that the dequant warps' 16-byte reads of consecutive rows are contiguous
-          tma_load_2d(smem + kOffPack + s * kPackBytes, &mapP, &b.full_ab[s], kt * (kBK / 2), prow);
-          tma_load_2d(smem + kOffPack + s * kPackBytes + kPackBytes / 2, &mapP, &b.full_ab[s], kt * (kBK / 2) + 16,
-                      prow);
+          mbar_arrive_expect_tx(&b.full_ab[s], kTokStage + kPackStage);
+          // One copy per operand and two K steps (a chunk past K reads as zeros): the token columns as
+          // 64-element chunks 2j, 2j+1 ([step][row][128 B], 128-byte swizzle), the packed bytes as 16-byte
+          // chunks 4j..4j+3 ([step][half][row][16 B], so the dequant warps' reads of consecutive rows are
+          // contiguous). Few large copies: the TMA unit's rate per SM goes with copies, not bytes.
+          tma_load_3d(smem + kOffTok + s * kTokStage, &mapA, &b.full_ab[s], 0, ti.row0, 2 * j);
+          tma_load_3d(smem + kOffPack + s * kPackStage, &mapP, &b.full_ab[s], 0, prow, 4 * j);
         }
       }
       // Drain: wait (bounded) for copies still in flight before the CTA may exit.
@@ -238,9 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       const uint8_t* sc = smem + kOffSc + sb * scbytes + r * KB + sc_blk;
       uint32_t va[kDeqCols];  // the converted step
-      auto convert = [&](int kt, int s, uint32_t* v) {
+      auto convert = [&](int kt, int s, uint32_t* v) {  // K step kt of the tile, from ring stage s
         const uint32_t sv = sc[kt * 2];
-        const uint8_t* src = smem + kOffPack + s * kPackBytes + pk_off;
+        const uint8_t* src = smem + kOffPack + s * kPackStage + (kt & 1) * kPackBytes + pk_off;
         if constexpr (kDeqCols == 16) {
           const uint4 pk = *reinterpret_cast<const uint4*>(src);
           const uint4 q0 = mx_dequant8_bf16(pk.x, sv), q1 = mx_dequant8_bf16(pk.y, sv);
@@ -254,9 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           v[0] = q0.x, v[1] = q0.y, v[2] = q0.z, v[3] = q0.w, v[4] = q1.x, v[5] = q1.y, v[6] = q1.z, v[7] = q1.w;
         }
       };
-      ok = wait_bar(&b.full_ab[it % kStages], (it / kStages) & 1, lim, abort_flag, a.status);
+      int gs = tc * SS;  // ring stage of the tile's first K step
+      ok = wait_bar(&b.full_ab[gs % kStages], (gs / kStages) & 1, lim, abort_flag, a.status);
       if (!ok) break;
-      convert(0, it % kStages, va);
+      convert(0, gs % kStages, va);
       for (int kt = 0; kt < KT; ++kt, ++it) {
         // Step it goes to TMEM stage it % kTStages once the MMAs of step it - kTStages are done; the
         // stage is handed to the MMA warp as soon as it is written, then the next step is converted
@@ -274,9 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&b.full_b[st]);
         if (kt + 1 < KT) {
-          ok = wait_bar(&b.full_ab[(it + 1) % kStages], ((it + 1) / kStages) & 1, lim, abort_flag, a.status);
+          gs = tc * SS + ((kt + 1) >> 1);
+          ok = wait_bar(&b.full_ab[gs % kStages], (gs / kStages) & 1, lim, abort_flag, a.status);
           if (!ok) break;
-          convert(kt + 1, (it + 1) % kStages, va);
+          convert(kt + 1, gs % kStages, va);
         }
       }
       if (!ok) break;
@@ -295,18 +297,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + ab * kAccCols;
         for (int kt = 0; kt < KT; ++kt, ++it) {
-          const int s = it % kStages, st = it % kTStages;
-          ok = wait_bar(&b.full_ab[s], (it / kStages) & 1, lim, abort_flag, a.status) &&
+          const int gs = tc * SS + (kt >> 1), s = gs % kStages, st = it % kTStages;
+          ok = wait_bar(&b.full_ab[s], (gs / kStages) & 1, lim, abort_flag, a.status) &&
                wait_bar(&b.full_b[st], (it / kTStages) & 1, lim, abort_flag, a.status);
           if (!ok) break;
           tc_fence_after();
           const uint32_t a_tmem = tmem_base + kAColBase + st * kAStageCols;
-          const uint32_t sbb = smem_u32(smem + kOffTok + s * kTokBytes);
+          const uint32_t sbb = smem_u32(smem + kOffTok + s * kTokStage + (kt & 1) * kTokBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
             umma_bf16_ts(d_tmem, a_tmem + kk * 8, smem_desc_k128(sbb + kk * 32), idesc, (kt | kk) ? 1u : 0u);
-          umma_commit(&b.empty[s]);
           umma_commit(&b.tfree[st]);
+          if ((kt & 1) || kt + 1 == KT) umma_commit(&b.empty[s]);  // the stage's K steps are done
         }
         if (!ok) break;
         umma_commit(&b.acc_full[ab]);
@@ -399,11 +401,12 @@ template <bool kGateUp>
 cudaError_t launch(const GemmArgs& a, const void* a_ptr, int sm_count, cudaStream_t st) {
   if (a.K % kBK || a.N % 64) return cudaErrorInvalidValue;
   CUtensorMap mapA, mapP;
-  if (!make_map_2d(&mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_ptr, a.K, a.total_rows, kBK, kTN,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  // tokens [total_rows][K] bf16 as 64-column chunks; packed weights [E*N][K/2] bytes as 16-byte chunks
+  if (!make_map_3d_chunks(&mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a_ptr, kBK, a.total_rows, a.K / kBK,
+                          (uint64_t)a.K * 2, kTN, 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  if (!make_map_2d(&mapP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.blocks, a.K / 2, (uint64_t)a.E * a.N, 16, kWM,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+  if (!make_map_3d_chunks(&mapP, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.blocks, 16, (uint64_t)a.E * a.N, a.K / 32,
+                          (uint64_t)a.K / 2, kWM, 4, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const size_t smem = smem_total(a.K);
   auto kern = grouped_mxfp4_gemm<kGateUp>;
