@@ -14,6 +14,7 @@ moe_status_t enqueue_layer(moe_ctx* h, const void* x, const float* rw, const flo
 cudaError_t raise_smem_limit(const void* func, size_t bytes);
 
 constexpr int kRouteTokPerBlock = 32;  // tokens per large-T router block (= one scatter chunk)
+constexpr int kRouteThreads = 512;     // threads of a large-T router block (16 warps)
 constexpr int kSmallT = 64;            // calls with T <= kSmallT route in one launch
 
 // Routing results written by the small-T router.

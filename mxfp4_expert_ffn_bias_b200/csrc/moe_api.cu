@@ -279,13 +279,13 @@ moe_status_t enqueue_route(moe_handle_t h, const void* x, const float* rw, const
     MOE_CHECK_CUDA(launch_pdl(split_router_kernel, dim3(nb), dim3(256), 0, st, rw, n, w.w3));
     MOE_CHECK_CUDA(cudaGetLastError());
   }
-  MOE_CHECK_CUDA(launch_pdl(route_mma_kernel, dim3(nchunk), dim3(256), route_mma_smem_bytes(E), st, xb, w.w3, rb, T, H,
+  MOE_CHECK_CUDA(launch_pdl(route_mma_kernel, dim3(nchunk), dim3(kRouteThreads), route_mma_smem_bytes(E), st, xb, w.w3, rb, T, H,
                             E, k, w.idx, w.w, w.counts, w.chunk_counts, w.xexp));
   MOE_CHECK_CUDA(cudaGetLastError());
   MOE_CHECK_CUDA(launch_pdl(route_scan_kernel, dim3(E), dim3(256), 0, st, w.counts, w.chunk_counts, nchunk, E,
                             w.chunk_base, w.offsets, w.mt_off, w.touched, w.n_touched));
   MOE_CHECK_CUDA(cudaGetLastError());
-  MOE_CHECK_CUDA(launch_pdl(route_scatter_kernel, dim3(nchunk), dim3(256), 0, st, w.idx, w.chunk_base, T, E, k, xb,
+  MOE_CHECK_CUDA(launch_pdl(route_scatter_kernel, dim3(nchunk, gather ? 4 : 1), dim3(256), 0, st, w.idx, w.chunk_base, T, E, k, xb,
                             H, gather ? 1 : 0, w.perm, w.x_perm));
   MOE_CHECK_CUDA(cudaGetLastError());
   return MOE_OK;

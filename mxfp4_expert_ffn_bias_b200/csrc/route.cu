@@ -9,11 +9,12 @@ namespace moe {
 
 // ---------------------------------------------------------------- router
 
-constexpr int kRouteWarps = 8;
-constexpr int kRouteTokPerWarp = 4;
+constexpr int kRouteWarps = 16;
+constexpr int kRouteTokPerWarp = 2;
 constexpr int kRouteTok = kRouteWarps * kRouteTokPerWarp;  // tokens per block (== kRouteTokPerBlock)
 constexpr int kMaxEJ = 8;                                  // experts per lane (E <= 256)
 static_assert(kRouteTok == kRouteTokPerBlock, "router chunk size");
+static_assert(kRouteWarps * 32 == kRouteThreads, "router block size");
 
 
 // k rounds of a warp-wide arg-max over the logits lg[j] of experts lane + 32j
@@ -108,7 +109,7 @@ __device__ __forceinline__ uint32_t absmax_bf16x8(uint4 v) {
 // load per row. K-group partial sums are added in shared memory in kg order.
 // Then, per token, top-k (ties: lower index), softmax over the k, the pair
 // counts per expert and per chunk, and the token's exponent c_t.
-__global__ void __launch_bounds__(256) route_mma_kernel(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(kRouteWarps * 32) route_mma_kernel(const uint16_t* __restrict__ x,
                                                         const uint16_t* __restrict__ w3, const float* __restrict__ rb,
                                                         int T, int H, int E, int k, int* __restrict__ idx_out,
                                                         float* __restrict__ w_out, int* __restrict__ counts,
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const uint16_t* __restri
   pdl_wait_and_trigger();
   extern __shared__ float smem[];
   const int NG = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
-  const int KG = 8 / NG;
+  const int KG = kRouteWarps / NG;
   float* red = smem;                                                 // [KG][32][E]
   uint32_t* s_amax = reinterpret_cast<uint32_t*>(red + (size_t)KG * 32 * E);  // [KG][32]
   int* s_cc = reinterpret_cast<int*>(s_amax + KG * 32);             // [E]
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(256) route_mma_kernel(const uint16_t* __restri
 
 size_t route_mma_smem_bytes(int E) {
   const int NG = E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8;
-  const int KG = 8 / NG;
+  const int KG = kRouteWarps / NG;
   return sizeof(float) * (size_t)KG * 32 * E + sizeof(uint32_t) * KG * 32 + sizeof(int) * 256;
 }
 
@@ -355,9 +356,10 @@ __global__ void __launch_bounds__(256) route_scan_kernel(const int* __restrict__
   }
 }
 
-// One block per router chunk (32 tokens): the stable rank of each pair among
-// the chunk's pairs with the same expert, plus chunk_base, is its permuted row.
-// Optionally copies the token's x row there (the A operand of the gate_up GEMM).
+// Blocks (chunk, y) for each router chunk (32 tokens): the stable rank of each pair among the chunk's
+// pairs with the same expert, plus chunk_base, is its permuted row; block y = 0 writes perm. Optionally the
+// blocks of a chunk copy its pairs' x rows there (the A operand of the gate_up GEMM), block y taking every
+// gridDim.y-th pair, one warp per row with all of the row's 16-byte loads in flight before its stores.
 __global__ void __launch_bounds__(256) route_scatter_kernel(const int* __restrict__ idx,
                                                             const int* __restrict__ chunk_base, int T, int E, int k,
                                                             const uint16_t* __restrict__ x, int H, int gather,
@@ -375,17 +377,30 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(const int* __restric
     int rank = 0;
     for (int j = 0; j < i; ++j) rank += (s_idx[j] == e);
     const int dest = chunk_base[(size_t)b * E + e] + rank;
-    perm[dest] = p0 + i;
+    if (blockIdx.y == 0) perm[dest] = p0 + i;
     s_dest[i] = dest;
   }
   if (!gather) return;
   __syncthreads();
-  const int nv = H / 8;
-#pragma unroll 4
-  for (int wi = tid; wi < P * nv; wi += blockDim.x) {
-    const int i = wi / nv, v = wi - i * nv;
-    reinterpret_cast<uint4*>(x_perm + (size_t)s_dest[i] * H)[v] =
-        reinterpret_cast<const uint4*>(x + (size_t)((p0 + i) / k) * H)[v];
+  const int lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const int nv = H / 8;  // 16-byte vectors per row
+  constexpr int kU = 12;
+  for (int i = (int)blockIdx.y + (int)gridDim.y * warp; i < P; i += (int)gridDim.y * nwarp) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)((p0 + i) / k) * H);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)s_dest[i] * H);
+    for (int v0 = 0; v0 < nv; v0 += 32 * kU) {
+      uint4 r[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int v = v0 + 32 * u + lane;
+        if (v < nv) r[u] = src[v];
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int v = v0 + 32 * u + lane;
+        if (v < nv) dst[v] = r[u];
+      }
+    }
   }
 }
 
@@ -626,20 +641,24 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(const uint16_t* _
 
 // ---------------------------------------------------------------- small-T router (one launch)
 
-// For T <= kSmallT, in three phases inside one launch:
-//  1. block (eg, hc) computes the partial logits of experts [8*eg, 8*eg+8)
-//     over hidden columns [hc*HC, (hc+1)*HC) for every token (and, for
-//     eg == 0, the partial max|x| of each token);
-//  2. the last block of expert group eg to finish (a ticket per group) sums
-//     the group's partials in hc order, adds the bias and writes its logits;
-//  3. the last group to finish (a second ticket) runs top-k and softmax for
-//     every token and the stable counting sort of all pairs in shared memory.
-// Each finishing block re-arms its ticket. The result does not depend on
-// which block finishes last.
+// For T <= kSmallT, in one launch:
+//  1. block (eg, hc), warp w: the partial logits of expert e = 8*eg + w over hidden columns
+//     [hc*HC, (hc+1)*HC) for every token. Lane l takes the column pairs 2l + 64i and accumulates
+//     eight tokens at once with fp32 FMAs, the loads of a batch all issued before its arithmetic;
+//     the warp then sums its lanes (butterfly). Warp 0 of group 0 also takes each token's partial
+//     max|x|.
+//  2. if T*E <= kRouteSingleMax, the last block of the grid to finish (one ticket) sums every
+//     (token, expert) partial in hc order, adds the bias and keeps the logits in shared memory.
+//     Otherwise the last block of each expert group (a ticket per group) writes its group's logits
+//     that way, and the last group to finish (a second ticket) goes on.
+//  3. that block runs top-k and softmax for every token and the stable counting sort of all pairs in
+//     shared memory.
+// Each finishing block re-arms its ticket. The result does not depend on which block finishes last.
+constexpr int kRouteSingleMax = 1024;
+
 size_t route_small_smem_bytes(int T, int E, int k, int HC) {
-  const size_t a = ((size_t)T * (HC + 2) * 2 + 15) / 16 * 16 + (size_t)8 * (HC + 1) * 4;
-  const size_t b = (size_t)T * E * 4 + (size_t)T * k * 4 + 3 * 260 * 4;
-  return a > b ? a : b;
+  (void)HC;
+  return (size_t)T * E * 4 + (size_t)T * k * 4 + 3 * 260 * 4 + (size_t)T * 4;
 }
 
 __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __restrict__ x,
@@ -657,88 +676,118 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
   pdl_wait_and_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h0 = hc * HC;
-  const int XS = HC + 2, WS = HC + 1;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(sm);
-  float* ws = reinterpret_cast<float*>(sm + ((size_t)T * XS * 2 + 15) / 16 * 16);
-  // (unrolled so that the loads of several iterations are in flight together)
-#pragma unroll 8
-  for (int i = tid; i < T * (HC / 2); i += blockDim.x) {
-    const int t = i / (HC / 2), c2 = i % (HC / 2);
-    *reinterpret_cast<uint32_t*>(xs + t * XS + 2 * c2) =
-        *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + 2 * c2);
-  }
-#pragma unroll 8
-  for (int i = tid; i < 8 * HC; i += blockDim.x) {
-    const int el = i / HC, c = i % HC, e = eg * 8 + el;
-    ws[el * WS + c] = (e < E) ? rw[(size_t)e * H + h0 + c] : 0.f;
-  }
-  __syncthreads();
-  // phase 1: outputs (t, el); `tpo` adjacent lanes share one output and split its columns
-  const int nout = T * 8;
-  int tpo = 1;
-  while (tpo < 32 && nout * tpo * 2 <= (int)blockDim.x) tpo *= 2;
-  for (int base = 0; base < nout * tpo; base += blockDim.x) {
-    const int li = base + tid;
-    const int oi = li / tpo, sub = li % tpo;  // tpo divides blockDim.x: a group never straddles two rounds
-    float acc = 0.f;
-    if (oi < nout) {
-      const int t = oi >> 3, el = oi & 7;
-      const uint16_t* xr = xs + t * XS;
-      const float* wr = ws + el * WS;
-      for (int c = sub; c < HC; c += tpo) acc = fmaf(bf16_bits_to_float(xr[c]), wr[c], acc);
-    }
-    for (int off = tpo >> 1; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (oi < nout && sub == 0) {
-      const int t = oi >> 3, e = eg * 8 + (oi & 7);
-      if (e < E) partial[((size_t)hc * T + t) * E + e] = acc;
-    }
-  }
-  if (eg == 0) {
-    for (int t = warp; t < T; t += 8) {
-      float m = 0.f;
-      for (int c = lane; c < HC; c += 32) m = fmaxf(m, fabsf(bf16_bits_to_float(xs[t * XS + c])));
+  const bool single = T * E <= kRouteSingleMax;
+
+  // phase 1
+  const int e1 = eg * 8 + warp;
+  if (e1 < E) {  // warp-uniform
+    const bool amax_warp = eg == 0 && warp == 0;
+    const float* wrow = rw + (size_t)e1 * H + h0 + 2 * lane;
+    const uint16_t* xcol = x + h0 + 2 * lane;
+    const int npair = HC / 64;
+    for (int t0 = 0; t0 < T; t0 += 8) {
+      const int nt = min(8, T - t0);
+      float acc[8], am[8];
 #pragma unroll
-      for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      if (lane == 0) pmax[(size_t)hc * T + t] = m;
+      for (int tt = 0; tt < 8; ++tt) acc[tt] = am[tt] = 0.f;
+      for (int i0 = 0; i0 < npair; i0 += 4) {
+        float2 wv[4];
+        uint32_t xv[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const bool ok = i0 + u < npair;
+          wv[u] = ok ? *reinterpret_cast<const float2*>(wrow + 64 * (i0 + u)) : make_float2(0.f, 0.f);
+#pragma unroll
+          for (int tt = 0; tt < 8; ++tt)
+            xv[u][tt] = (ok && tt < nt)
+                            ? *reinterpret_cast<const uint32_t*>(xcol + (size_t)(t0 + tt) * H + 64 * (i0 + u))
+                            : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int tt = 0; tt < 8; ++tt) {
+            const float xa = bf16_bits_to_float(xv[u][tt] & 0xFFFFu), xb = bf16_bits_to_float(xv[u][tt] >> 16);
+            acc[tt] = fmaf(xa, wv[u].x, acc[tt]);
+            acc[tt] = fmaf(xb, wv[u].y, acc[tt]);
+            am[tt] = fmaxf(am[tt], fmaxf(fabsf(xa), fabsf(xb)));
+          }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 8; ++tt)
+#pragma unroll
+        for (int off = 16; off; off >>= 1) acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], off);
+      if (amax_warp) {
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt)
+#pragma unroll
+          for (int off = 16; off; off >>= 1) am[tt] = fmaxf(am[tt], __shfl_xor_sync(0xffffffffu, am[tt], off));
+      }
+#pragma unroll
+      for (int tt = 0; tt < 8; ++tt) {
+        if (lane == tt && tt < nt) {
+          partial[((size_t)hc * T + t0 + tt) * E + e1] = acc[tt];
+          if (amax_warp) pmax[(size_t)hc * T + t0 + tt] = am[tt];
+        }
+      }
     }
   }
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    s_last = atomicAdd(&ticket[1 + eg], 1) == nHC - 1;
+    s_last = single ? atomicAdd(&ticket[0], 1) == nEG * nHC - 1 : atomicAdd(&ticket[1 + eg], 1) == nHC - 1;
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
 
-  // phase 2: the group's logits, partials summed in hc order
-  for (int oi = tid; oi < nout; oi += blockDim.x) {
-    const int t = oi >> 3, e = eg * 8 + (oi & 7);
-    if (e >= E) continue;
-    float v = 0.f;
-#pragma unroll 8
-    for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
-    logits[(size_t)t * E + e] = v + rb[e];
-  }
-  __syncthreads();
-  if (tid == 0) {
-    ticket[1 + eg] = 0;  // re-arm for the next call
-    __threadfence();
-    s_last = atomicAdd(&ticket[0], 1) == nEG - 1;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-
-  // phase 3 (last group): top-k, softmax, counting sort
-  float* lg = reinterpret_cast<float*>(sm);     // [T][E]
+  float* lg = reinterpret_cast<float*>(sm);                 // [T][E]
   int* s_idx = reinterpret_cast<int*>(lg + (size_t)T * E);  // [T*k]
-  int* s_cnt = s_idx + T * k;                   // [E]
-  int* s_off = s_cnt + 260;                     // [E+1]
-  int* s_mt = s_off + 260;                      // [E+1]
+  int* s_cnt = s_idx + T * k;                               // [E]
+  int* s_off = s_cnt + 260;                                 // [E+1]
+  int* s_mt = s_off + 260;                                  // [E+1]
+  float* s_pm = reinterpret_cast<float*>(s_mt + 260);       // [T]
+  if (single) {
+    // phase 2: every logit, partials summed in hc order
+    for (int oi = tid; oi < T * E; oi += blockDim.x) {
+      const int t = oi / E, e = oi - t * E;
+      float v = 0.f;
 #pragma unroll 8
-  for (int i = tid; i < T * E; i += blockDim.x) lg[i] = __ldcg(&logits[i]);
+      for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
+      lg[oi] = v + rb[e];
+    }
+  } else {
+    // phase 2: the group's logits, partials summed in hc order
+    const int nout = T * 8;
+    for (int oi = tid; oi < nout; oi += blockDim.x) {
+      const int t = oi >> 3, e = eg * 8 + (oi & 7);
+      if (e >= E) continue;
+      float v = 0.f;
+#pragma unroll 8
+      for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
+      logits[(size_t)t * E + e] = v + rb[e];
+    }
+    __syncthreads();
+    if (tid == 0) {
+      ticket[1 + eg] = 0;  // re-arm for the next call
+      __threadfence();
+      s_last = atomicAdd(&ticket[0], 1) == nEG - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+#pragma unroll 8
+    for (int i = tid; i < T * E; i += blockDim.x) lg[i] = __ldcg(&logits[i]);
+  }
+  for (int t = tid; t < T; t += blockDim.x) {
+    float m = 0.f;
+    for (int h = 0; h < nHC; ++h) m = fmaxf(m, __ldcg(&pmax[(size_t)h * T + t]));
+    s_pm[t] = m;
+  }
+  for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
   __syncthreads();
+
+  // phase 3: top-k, softmax, counting sort
   const int EJ = (E + 31) / 32;
   for (int t = warp; t < T; t += 8) {
     float l[kMaxEJ];
@@ -750,41 +799,44 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     int sele[8];
     float selv[8], w[8];
     warp_topk(l, EJ, E, k, sele, selv);
-    float m = 0.f;
-    for (int h = lane; h < nHC; h += 32) m = fmaxf(m, __ldcg(&pmax[(size_t)h * T + t]));
+    if (lane == 0) softmax_k(selv, k, w);
+    if (lane < k) {  // lane s publishes slot s (register arrays indexed by unrolled s only)
 #pragma unroll
-    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    if (lane == 0) {
-      softmax_k(selv, k, w);
-      o.xexp[t] = token_exponent(m);
-      for (int s = 0; s < k; ++s) {
-        o.idx[t * k + s] = sele[s];
-        o.w[t * k + s] = w[s];
-        s_idx[t * k + s] = sele[s];
+      for (int s = 0; s < 8; ++s) {
+        if (s == lane) {
+          o.idx[t * k + s] = sele[s];
+          s_idx[t * k + s] = sele[s];
+          atomicAdd(&s_cnt[sele[s]], 1);  // integer counts: the same whatever the order
+        }
       }
+    }
+    if (lane == 0) {
+      o.xexp[t] = token_exponent(s_pm[t]);
+      for (int s = 0; s < k; ++s) o.w[t * k + s] = w[s];
     }
   }
   __syncthreads();
   const int Tk = T * k;
-  for (int e = tid; e < E; e += blockDim.x) {
-    int c = 0;
-    for (int p = 0; p < Tk; ++p) c += (s_idx[p] == e);
-    s_cnt[e] = c;
-    o.counts[e] = c;
-  }
-  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) o.counts[e] = s_cnt[e];
   prefix_counts(s_cnt, E, s_off, s_mt);
   __syncthreads();
   for (int i = tid; i <= E; i += blockDim.x) {
     o.offsets[i] = s_off[i];
     o.mt_off[i] = s_mt[i];
   }
-  if (tid == 0) {
+  if (warp == 0) {  // touched experts in increasing order
     int n = 0;
-    for (int j = 0; j < E; ++j)
-      if (s_cnt[j] > 0) o.touched[n++] = j;
-    *o.n_touched = n;
-    ticket[0] = 0;  // re-arm for the next call
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const bool on = e < E && s_cnt[e] > 0;
+      const unsigned m = __ballot_sync(0xffffffffu, on);
+      if (on) o.touched[n + __popc(m & ((1u << lane) - 1u))] = e;
+      n += __popc(m);
+    }
+    if (lane == 0) {
+      *o.n_touched = n;
+      ticket[0] = 0;  // re-arm for the next call
+    }
   }
   for (int p = tid; p < Tk; p += blockDim.x) {
     const int e = s_idx[p];
