@@ -17,45 +17,77 @@ static_assert(kRouteTok == kRouteTokPerBlock, "router chunk size");
 static_assert(kRouteWarps * 32 == kRouteThreads, "router block size");
 
 
+// Unsigned key with the order of the float values (-0 and +0 equal; no NaN): nonzero for every value.
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.f);  // -0 + +0 = +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // k rounds of a warp-wide arg-max over the logits lg[j] of experts lane + 32j
-// (ties: lower expert index). Every lane ends with the same sele/selv.
-__device__ __forceinline__ void warp_topk(const float (&lg)[kMaxEJ], int EJ, int E, int k, int* sele, float* selv) {
+// (ties: lower expert index). Each round: every lane's best untaken expert
+// (ascending j, strict comparison: the lower index wins a tie), then the warp's
+// largest key (redux max) and, among the lanes holding it, the lowest expert
+// index (redux min). Every lane ends with the same sele/selv. The rounds are
+// unrolled (k <= 8) so that sele/selv stay in registers.
+__device__ __forceinline__ void warp_topk(const float (&lg)[kMaxEJ], int EJ, int E, int k, int (&sele)[8],
+                                          float (&selv)[8]) {
   const int lane = threadIdx.x & 31;
-  unsigned taken = 0;
-  for (int s = 0; s < k; ++s) {
+  uint32_t key[kMaxEJ];
+#pragma unroll
+  for (int j = 0; j < kMaxEJ; ++j) key[j] = (j < EJ && lane + 32 * j < E) ? order_key(lg[j]) : 0u;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    if (s >= k) break;
+    uint32_t bk = 0u, be = 0xFFFFFFFFu;
     float bv = -INFINITY;
-    int be = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < kMaxEJ; ++j) {
-      const int e = lane + 32 * j;
-      if (j < EJ && e < E && !(taken & (1u << j)) && (lg[j] > bv || (lg[j] == bv && e < be))) {
+      if (key[j] > bk) {
+        bk = key[j];
+        be = (uint32_t)(lane + 32 * j);
         bv = lg[j];
-        be = e;
       }
     }
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t me = __reduce_min_sync(0xffffffffu, bk == mk ? be : 0xFFFFFFFFu);
+    selv[s] = __shfl_sync(0xffffffffu, bv, (int)(me & 31u));
+    sele[s] = (int)me;
+    if ((me & 31u) == (uint32_t)lane) {
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
+      for (int j = 0; j < kMaxEJ; ++j)
+        if ((uint32_t)j == (me >> 5)) key[j] = 0u;  // taken
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    selv[s] = bv;
-    sele[s] = be;
   }
 }
 
-// Softmax over the k selected logits (fp32, max subtracted), as the weights w_s.
-__device__ __forceinline__ void softmax_k(const float* selv, int k, float* w) {
+// sum_{h < n} p[h * stride] in h order (__ldcg), the loads of each batch of 16 issued together.
+__device__ __forceinline__ float sum_strided_ldcg(const float* p, size_t stride, int n) {
+  float v = 0.f;
+  for (int h0 = 0; h0 < n; h0 += 16) {
+    float r[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) r[u] = h0 + u < n ? __ldcg(p + (size_t)(h0 + u) * stride) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 16; ++u)
+      if (h0 + u < n) v += r[u];
+  }
+  return v;
+}
+
+// Softmax over the k selected logits (fp32, max subtracted), as the weights w_s (k <= 8, unrolled).
+__device__ __forceinline__ void softmax_k(const float (&selv)[8], int k, float (&w)[8]) {
   float z = 0.f;
-  for (int s = 0; s < k; ++s) {
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    if (s >= k) break;
     w[s] = expf(selv[s] - selv[0]);
     z += w[s];
   }
-  for (int s = 0; s < k; ++s) w[s] /= z;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    if (s >= k) break;
+    w[s] /= z;
+  }
 }
 
 // Exponent c_t with max|x_t| * 2^-c_t in [2^14, 2^15) (0 for an all-zero row).
@@ -232,7 +264,9 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_mma_kernel(const uint1
       uint32_t m = 0;
       for (int kk = 0; kk < KG; ++kk) m = max(m, s_amax[kk * 32 + tl]);
       softmax_k(selv, k, w);
-      for (int s = 0; s < k; ++s) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        if (s >= k) break;
         idx_out[t * k + s] = sele[s];
         w_out[t * k + s] = w[s];
         atomicAdd(&counts[sele[s]], 1);  // integer counts: the same whatever the order
@@ -496,24 +530,42 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(const uint16_t* _
   const int h0 = (int)rank * HS;
 
   // stage this CTA's columns, transposed; consecutive threads take consecutive tokens / experts so that
-  // the shared-memory stores are conflict-free (unrolled so that several loads are in flight)
-#pragma unroll 4
-  for (int i = tid; i < Tp * (HS / 2); i += nthr) {
-    const int c2 = i / Tp, t = i - c2 * Tp;
-    uint32_t v = 0;
-    if (t < T) v = *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + 2 * c2);
-    xT[(2 * c2) * Tp + t] = bf16_bits_to_float(v & 0xFFFF);
-    xT[(2 * c2 + 1) * Tp + t] = bf16_bits_to_float(v >> 16);
+  // the shared-memory stores are conflict-free (batches of 4 loads per thread issued together)
+  constexpr int kB = 4;
+  for (int i0 = tid; i0 < Tp * (HS / 2); i0 += kB * nthr) {
+    uint32_t v[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = i0 + u * nthr, c2 = i / Tp, t = i - c2 * Tp;
+      v[u] = (i < Tp * (HS / 2) && t < T) ? *reinterpret_cast<const uint32_t*>(x + (size_t)t * H + h0 + 2 * c2) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = i0 + u * nthr, c2 = i / Tp, t = i - c2 * Tp;
+      if (i < Tp * (HS / 2)) {
+        xT[(2 * c2) * Tp + t] = bf16_bits_to_float(v[u] & 0xFFFF);
+        xT[(2 * c2 + 1) * Tp + t] = bf16_bits_to_float(v[u] >> 16);
+      }
+    }
   }
-#pragma unroll 4
-  for (int i = tid; i < Ep * (HS / 4); i += nthr) {
-    const int c4 = i / Ep, e = i - c4 * Ep;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (e < E) v = *reinterpret_cast<const float4*>(rw + (size_t)e * H + h0 + 4 * c4);
-    wT[(4 * c4) * Ep + e] = v.x;
-    wT[(4 * c4 + 1) * Ep + e] = v.y;
-    wT[(4 * c4 + 2) * Ep + e] = v.z;
-    wT[(4 * c4 + 3) * Ep + e] = v.w;
+  for (int i0 = tid; i0 < Ep * (HS / 4); i0 += kB * nthr) {
+    float4 v[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = i0 + u * nthr, c4 = i / Ep, e = i - c4 * Ep;
+      v[u] = (i < Ep * (HS / 4) && e < E) ? *reinterpret_cast<const float4*>(rw + (size_t)e * H + h0 + 4 * c4)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const int i = i0 + u * nthr, c4 = i / Ep, e = i - c4 * Ep;
+      if (i < Ep * (HS / 4)) {
+        wT[(4 * c4) * Ep + e] = v[u].x;
+        wT[(4 * c4 + 1) * Ep + e] = v[u].y;
+        wT[(4 * c4 + 2) * Ep + e] = v[u].z;
+        wT[(4 * c4 + 3) * Ep + e] = v[u].w;
+      }
+    }
   }
   __syncthreads();
   // partial max|x| per token over this CTA's columns
@@ -600,7 +652,9 @@ __global__ void __launch_bounds__(512, 1) route_cluster_kernel(const uint16_t* _
     if (lane == 0) {
       softmax_k(selv, k, w);
       o.xexp[t] = token_exponent(m);
-      for (int s = 0; s < k; ++s) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        if (s >= k) break;
         o.idx[t * k + s] = sele[s];
         o.w[t * k + s] = w[s];
         st_cluster_u32(map_to_cta(s_sel + t * k + s, 0u), (uint32_t)sele[s]);
@@ -747,14 +801,18 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
   int* s_off = s_cnt + 260;                                 // [E+1]
   int* s_mt = s_off + 260;                                  // [E+1]
   float* s_pm = reinterpret_cast<float*>(s_mt + 260);       // [T]
+  for (int t = warp; t < T; t += 8) {  // each token's max|x|: lane h takes chunk h, then a warp max
+    float m = 0.f;
+    for (int h = lane; h < nHC; h += 32) m = fmaxf(m, __ldcg(&pmax[(size_t)h * T + t]));
+#pragma unroll
+    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) s_pm[t] = m;
+  }
   if (single) {
     // phase 2: every logit, partials summed in hc order
     for (int oi = tid; oi < T * E; oi += blockDim.x) {
       const int t = oi / E, e = oi - t * E;
-      float v = 0.f;
-#pragma unroll 8
-      for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
-      lg[oi] = v + rb[e];
+      lg[oi] = sum_strided_ldcg(partial + (size_t)t * E + e, (size_t)T * E, nHC) + rb[e];
     }
   } else {
     // phase 2: the group's logits, partials summed in hc order
@@ -762,10 +820,7 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     for (int oi = tid; oi < nout; oi += blockDim.x) {
       const int t = oi >> 3, e = eg * 8 + (oi & 7);
       if (e >= E) continue;
-      float v = 0.f;
-#pragma unroll 8
-      for (int h = 0; h < nHC; ++h) v += __ldcg(&partial[((size_t)h * T + t) * E + e]);
-      logits[(size_t)t * E + e] = v + rb[e];
+      logits[(size_t)t * E + e] = sum_strided_ldcg(partial + (size_t)t * E + e, (size_t)T * E, nHC) + rb[e];
     }
     __syncthreads();
     if (tid == 0) {
@@ -778,11 +833,6 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     __threadfence();
 #pragma unroll 8
     for (int i = tid; i < T * E; i += blockDim.x) lg[i] = __ldcg(&logits[i]);
-  }
-  for (int t = tid; t < T; t += blockDim.x) {
-    float m = 0.f;
-    for (int h = 0; h < nHC; ++h) m = fmaxf(m, __ldcg(&pmax[(size_t)h * T + t]));
-    s_pm[t] = m;
   }
   for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
   __syncthreads();
@@ -812,7 +862,11 @@ __global__ void __launch_bounds__(256) route_small_kernel(const uint16_t* __rest
     }
     if (lane == 0) {
       o.xexp[t] = token_exponent(s_pm[t]);
-      for (int s = 0; s < k; ++s) o.w[t * k + s] = w[s];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        if (s >= k) break;
+        o.w[t * k + s] = w[s];
+      }
     }
   }
   __syncthreads();
@@ -875,13 +929,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     const long long t = i / H4;
     const int j4 = (int)(i % H4);
     const float4* src = reinterpret_cast<const float4*>(slot + (size_t)t * k * H) + j4;
-    float4 a = src[0];
-    for (int s = 1; s < k; ++s) {
-      const float4 b = src[(size_t)s * H4];
-      a.x += b.x;
-      a.y += b.y;
-      a.z += b.z;
-      a.w += b.w;
+    float4 b[8];  // k <= 8: every slot's load in flight together, then the sum in slot order
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < k) b[s] = src[(size_t)s * H4];
+    float4 a = b[0];
+#pragma unroll
+    for (int s = 1; s < 8; ++s) {
+      if (s >= k) break;
+      a.x += b[s].x;
+      a.y += b[s].y;
+      a.z += b[s].z;
+      a.w += b[s].w;
     }
     uint2 o;
     o.x = pack_bf16x2(a.x, a.y);
