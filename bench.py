@@ -57,7 +57,7 @@ def parse_args():
     ap.add_argument("--path", type=int, default=0, help="0 auto, 1 decode GEMV, 2 grouped GEMM")
     ap.add_argument("--decode-kernel", type=int, default=-1,
                     help="decode GEMV engine: 0 CUDA-core FMA, 1 warp MMA per row slab, 2 persistent warp MMA, "
-                         "-1 per stage (gate_up 1, down 2)")
+                         "-1 default (1 for both stages)")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill side measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     return ap.parse_args()

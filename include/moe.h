@@ -68,8 +68,8 @@ enum moe_option {
   MOE_OPT_DECODE_KERNEL = 5, /* decode-path GEMV engine: 0 = CUDA-core mixed-precision FMAs, 1 = m16n8k16
                                 warp MMAs, one block per slab of an expert's rows, 2 = the same warp MMAs in
                                 persistent CTAs whose warps stream their rows through asynchronous-copy
-                                rings, -1 (default) = 1 for gate_up and 2 for down (measured fastest on
-                                B200 for the GPT-OSS decode shapes). All compute the same products in fp32. */
+                                rings, -1 (default) = 1 for both stages (measured fastest on B200 for the
+                                GPT-OSS decode shapes). All compute the same products in fp32. */
   MOE_OPT_STAGE_EVENTS = 4   /* n > 0: record CUDA events on each call's stream before the first kernel and
                                 after each of the MOE_NUM_STAGES stages, for up to n calls (a ring; read
                                 and reset with moe_stage_times). 0 = off. */

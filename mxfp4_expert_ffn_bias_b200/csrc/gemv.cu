@@ -27,6 +27,49 @@ constexpr int kGemvUnroll = 4;     // MX blocks in flight per lane
 
 size_t gemv_smem_bytes(int C) { return (size_t)kGemvTok * C * sizeof(uint16_t); }
 
+// Stages nrows token rows of C columns into xs (f16, row pitch CP); rows m >= mc are zero. gate_up: row m
+// is x[perm[row_base + m0 + m] / k] * 2^-c_t; down: the f16 activation row row_base + m0 + m. Each thread
+// takes kSB 16-byte units per batch and issues the batch's loads together, level by level (pair index,
+// then c_t, then the row), so that a batch costs one round trip per level, not one per unit.
+template <bool kGateUp>
+__device__ __forceinline__ void stage_tokens(const GemvArgs& a, int row_base, int m0, int mc, int nrows, int C,
+                                             int CP, uint16_t* xs, int tid, int nthr) {
+  constexpr int kSB = 4;
+  const int nv = C / 8, n = nrows * nv;
+  for (int i0 = tid; i0 < n; i0 += kSB * nthr) {
+    int tok[kSB];
+    float sc[kSB];
+    uint4 raw[kSB];
+#pragma unroll
+    for (int u = 0; u < kSB; ++u) {
+      const int i = i0 + u * nthr, m = i / nv;
+      tok[u] = -1;
+      if (i < n && m < mc) tok[u] = kGateUp ? a.perm[row_base + m0 + m] / a.k : row_base + m0 + m;
+    }
+#pragma unroll
+    for (int u = 0; u < kSB; ++u) sc[u] = (kGateUp && tok[u] >= 0) ? exp2_int(-a.xexp[tok[u]]) : 1.f;
+#pragma unroll
+    for (int u = 0; u < kSB; ++u) {
+      const int i = i0 + u * nthr, c8 = i - (i / nv) * nv;
+      raw[u] = tok[u] >= 0 ? reinterpret_cast<const uint4*>(a.xin + (size_t)tok[u] * C)[c8] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kSB; ++u) {
+      const int i = i0 + u * nthr, m = i / nv, c8 = i - m * nv;
+      if (i >= n) continue;
+      uint4 v = raw[u];
+      if (kGateUp && tok[u] >= 0) {  // x * 2^-c_t in f16
+        const uint4 r = raw[u];
+        v.x = pack_f16x2(bf16_bits_to_float(r.x & 0xFFFF) * sc[u], bf16_bits_to_float(r.x >> 16) * sc[u]);
+        v.y = pack_f16x2(bf16_bits_to_float(r.y & 0xFFFF) * sc[u], bf16_bits_to_float(r.y >> 16) * sc[u]);
+        v.z = pack_f16x2(bf16_bits_to_float(r.z & 0xFFFF) * sc[u], bf16_bits_to_float(r.z >> 16) * sc[u]);
+        v.w = pack_f16x2(bf16_bits_to_float(r.w & 0xFFFF) * sc[u], bf16_bits_to_float(r.w >> 16) * sc[u]);
+      }
+      reinterpret_cast<uint4*>(xs + (size_t)m * CP)[c8] = v;
+    }
+  }
+}
+
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -272,7 +315,16 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(GemvArgs a) {
   {
     const uint4* src = reinterpret_cast<const uint4*>(a.scales + ((size_t)e * R + r0) * KB);
     uint4* dst = reinterpret_cast<uint4*>(scs);
-    for (int i = tid; i < rows_here * KB / 16; i += kMmaWarps * 32) dst[i] = src[i];
+    const int n = rows_here * KB / 16;
+    for (int i0 = tid; i0 < n; i0 += 4 * kMmaWarps * 32) {  // four loads per thread in flight
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + u * kMmaWarps * 32 < n) v[u] = src[i0 + u * kMmaWarps * 32];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + u * kMmaWarps * 32 < n) dst[i0 + u * kMmaWarps * 32] = v[u];
+    }
   }
 
   for (int m0 = 0; m0 < Me; m0 += kGemvTok) {
@@ -283,22 +335,7 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(GemvArgs a) {
       else mma_load<false>(A, w0p, w1p, 0, KB);
     }
     __syncthreads();
-    for (int i = tid; i < mc * (C / 8); i += kMmaWarps * 32) {
-      const int m = i / (C / 8), c8 = i % (C / 8);
-      uint4 v;
-      if (kGateUp) {  // tokens in f16, scaled by 2^-c_t
-        const int t = a.perm[row_base + m0 + m] / a.k;
-        const float sc = exp2_int(-a.xexp[t]);
-        const uint4 raw = reinterpret_cast<const uint4*>(a.xin + (size_t)t * C)[c8];
-        v.x = pack_f16x2(bf16_bits_to_float(raw.x & 0xFFFF) * sc, bf16_bits_to_float(raw.x >> 16) * sc);
-        v.y = pack_f16x2(bf16_bits_to_float(raw.y & 0xFFFF) * sc, bf16_bits_to_float(raw.y >> 16) * sc);
-        v.z = pack_f16x2(bf16_bits_to_float(raw.z & 0xFFFF) * sc, bf16_bits_to_float(raw.z >> 16) * sc);
-        v.w = pack_f16x2(bf16_bits_to_float(raw.w & 0xFFFF) * sc, bf16_bits_to_float(raw.w >> 16) * sc);
-      } else {
-        v = reinterpret_cast<const uint4*>(a.xin + (size_t)(row_base + m0 + m) * C)[c8];
-      }
-      reinterpret_cast<uint4*>(xs + (size_t)m * CP)[c8] = v;
-    }
+    stage_tokens<kGateUp>(a, row_base, m0, mc, mc, C, CP, xs, tid, kMmaWarps * 32);
     __syncthreads();
     if (!warp_on) continue;
     const bool has_tok = g < mc;
@@ -621,30 +658,12 @@ __global__ void __launch_bounds__(kVThreads, 1) gemv_v_kernel(GemvArgs a) {
       if (e != st_e || m0 != st_m0) {  // (re)stage the pass's tokens in f16
         ok = cta_sync(b, cons_ph, lim, a.status);
         if (!ok) break;
-        const int nv = C / 8;
         if (tid < mc) {
           const int pr = a.perm[row_base + m0 + tid];
           s_pair[tid] = pr;
           s_scl[tid] = kGateUp ? exp2_int(a.xexp[pr / a.k]) : a.wroute[pr];
         }
-        for (int i = tid; i < tpp * nv; i += kVThreads) {
-          const int m = i / nv, c8 = i - m * nv;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (m < mc) {
-            if (kGateUp) {  // x * 2^-c_t in f16
-              const int tok = a.perm[row_base + m0 + m] / a.k;
-              const float sc = exp2_int(-a.xexp[tok]);
-              const uint4 raw = reinterpret_cast<const uint4*>(a.xin + (size_t)tok * C)[c8];
-              v.x = pack_f16x2(bf16_bits_to_float(raw.x & 0xFFFF) * sc, bf16_bits_to_float(raw.x >> 16) * sc);
-              v.y = pack_f16x2(bf16_bits_to_float(raw.y & 0xFFFF) * sc, bf16_bits_to_float(raw.y >> 16) * sc);
-              v.z = pack_f16x2(bf16_bits_to_float(raw.z & 0xFFFF) * sc, bf16_bits_to_float(raw.z >> 16) * sc);
-              v.w = pack_f16x2(bf16_bits_to_float(raw.w & 0xFFFF) * sc, bf16_bits_to_float(raw.w >> 16) * sc);
-            } else {
-              v = reinterpret_cast<const uint4*>(a.xin + (size_t)(row_base + m0 + m) * C)[c8];
-            }
-          }
-          reinterpret_cast<uint4*>(xs + (size_t)m * CP)[c8] = v;
-        }
+        stage_tokens<kGateUp>(a, row_base, m0, mc, tpp, C, CP, xs, tid, kVThreads);
         ok = cta_sync(b, cons_ph, lim, a.status);
         if (!ok) break;
         st_e = e;

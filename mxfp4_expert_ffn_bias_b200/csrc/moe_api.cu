@@ -352,7 +352,7 @@ moe_status_t enqueue_forward(moe_handle_t h, const void* x, const float* rw, con
     g.act_out = nullptr;
     g.R = H;
     g.C = I;
-    MOE_CHECK_CUDA(launch_gemv_down(g, max_touched, h->gemv_variant < 0 ? 2 : h->gemv_variant, h->sm_count, st));
+    MOE_CHECK_CUDA(launch_gemv_down(g, max_touched, h->gemv_variant < 0 ? 1 : h->gemv_variant, h->sm_count, st));
   } else {
     if (rec) MOE_CHECK_CUDA(cudaEventRecord(ev[1], st));
     GemmArgs g{};
