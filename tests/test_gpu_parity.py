@@ -127,6 +127,41 @@ def test_route_topk_softmax_and_permutation(moe, name):
     assert np.array_equal(offs.cpu().numpy(), np.concatenate([[0], np.cumsum(counts)]))
 
 
+# Token counts that reach each router kernel and each of its branches: the small-T router with one ticket
+# (T*E <= 1024) and with a ticket per expert group (above), the 16-CTA cluster router (T*E >= 2048, T <= 64),
+# and the large-T tensor-core router with 1, 2, 4 and 8 expert groups per block (E = 32, 64, 128, 256);
+# E = 256 with top-8 also runs every unrolled top-k round and eight experts per lane.
+_WIDE256 = Config("wide-256", T=96, H=256, I=256, E=256, k=8, scale_lo=119, scale_hi=123, router_bias="normal")
+_WIDE64 = Config("wide-64", T=80, H=512, I=256, E=64, k=4, scale_lo=119, scale_hi=123, router_bias="normal")
+ROUTE_SIZES = [("gpt-oss-20b-decode", 40), ("gpt-oss-20b-decode", 64), ("gpt-oss-120b-decode", 12),
+               ("gpt-oss-120b-decode", 100), (_WIDE256, 4), (_WIDE256, 6), (_WIDE256, 96), (_WIDE64, 80)]
+
+
+@pytest.mark.parametrize("name,T", ROUTE_SIZES, ids=[f"{getattr(c, 'name', c)}-T{t}" for c, t in ROUTE_SIZES])
+def test_route_branches_by_size(moe, name, T):
+    cfg = cfg_of(name)
+    inp = inputs_for(name, T=T)
+    dev = to_device(inp)
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
+    try:
+        idx = torch.empty((T, cfg.k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, cfg.k), dtype=torch.float32, device="cuda")
+        perm = torch.empty(T * cfg.k, dtype=torch.int32, device="cuda")
+        offs = torch.empty(cfg.E + 1, dtype=torch.int32, device="cuda")
+        for _ in range(2):  # twice: the tickets must be re-armed by the first call
+            moe.moe_debug_route(h, dev["x"], dev["router_w"], dev["router_b"], T, idx, w, perm, offs)
+            torch.cuda.synchronize()
+            lg = oracle.router_logits(inp["x"], inp["router_w"], inp["router_b"])
+            ref_idx, ref_w = oracle.topk_softmax(lg, cfg.k)
+            assert np.array_equal(idx.cpu().numpy(), ref_idx)
+            assert np.abs(w.cpu().numpy() - ref_w).max() <= 1e-5
+            assert np.array_equal(perm.cpu().numpy(), np.argsort(ref_idx.ravel(), kind="stable"))
+            counts = np.bincount(ref_idx.ravel(), minlength=cfg.E)
+            assert np.array_equal(offs.cpu().numpy(), np.concatenate([[0], np.cumsum(counts)]))
+    finally:
+        moe.moe_destroy(h)
+
+
 # ---------------------------------------------------------------- whole layer
 
 
@@ -194,6 +229,13 @@ def test_all_experts_selected_and_single_expert(moe, path, variant):
 def test_gpt_oss_20b_decode(moe, path, variant):
     got, ref, _ = _run_layer(moe, "gpt-oss-20b-decode", path, variant=variant)
     assert_parity(got, ref, f"20b decode path={path} variant={variant}")
+
+
+def test_gpt_oss_20b_decode_40_tokens_sampled(moe):
+    # 40 x 32 logits: the small-T router with a ticket per expert group, then the default decode engines
+    tokens = [0, 1, 13, 22, 38, 39]
+    got, ref, _ = _run_layer(moe, "gpt-oss-20b-decode", 1, T=40, tokens=tokens)
+    assert_parity(got, ref, "20b decode T=40")
 
 
 @pytest.mark.parametrize("path,variant", PATHS)
