@@ -109,8 +109,8 @@ _GEMV_TU = ["mxfp4_expert_ffn_bias_b200/csrc/gemv.cu", "mxfp4_expert_ffn_bias_b2
             "include/moe.h"]
 _GEMM_TU = ["mxfp4_expert_ffn_bias_b200/csrc/gemm_sm100.cu"] + _GEMV_TU[1:]
 TRAFFIC = {
-    # profiles/decode-kernels_gpt-oss-20b-decode.md: 194.27 MB read + 3.90 MB written
-    ("moe::gemv_mma_kernel<true>", "gpt-oss-20b-decode"): {"bytes": 198171648, "files": _GEMV_TU, "hash": "64070750bd453ab3"},
+    # profiles/decode-kernels_gpt-oss-20b-decode.md: 194.24 MB read + 5.55 MB written
+    ("moe::gemv_mma_kernel<true>", "gpt-oss-20b-decode"): {"bytes": 199787520, "files": _GEMV_TU, "hash": "ba40c91127ef9c21"},
     # profiles/prefill-kernels_gpt-oss-20b-prefill.md: 376.81 MB read + 82.16 MB written
     ("moe::grouped_mxfp4_gemm<true>", "gpt-oss-20b-prefill"): {"bytes": 458969088, "files": _GEMM_TU, "hash": "2d304a3f9878b4a8"},
 }

@@ -212,11 +212,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(GemvArgs a) {
 #define MOE_GEMV_UNROLL 8
 #endif
 constexpr int kMmaUnroll = MOE_GEMV_UNROLL;  // MX blocks per pipeline group (two groups in flight)
-#ifndef MOE_GEMV_WARPS
-#define MOE_GEMV_WARPS 6
-#endif
-constexpr int kMmaWarps = MOE_GEMV_WARPS;    // warps per block (measured best of 4, 6, 8 on the gpt-oss decode shapes)
-constexpr int kMmaRows = 16 * kMmaWarps;  // weight rows per block
+// Warps per block, per stage (measured best of 4, 6, 8 on the gpt-oss decode shapes: 6 for gate_up, 8 for
+// down); a block holds 16 weight rows per warp.
+constexpr int kMmaWarpsGateUp = 6;
+constexpr int kMmaWarpsDown = 8;
+__host__ __device__ constexpr int mma_warps(bool gate_up) { return gate_up ? kMmaWarpsGateUp : kMmaWarpsDown; }
 
 __device__ __forceinline__ uint32_t ldg_u32(const void* p) {
   uint32_t v;
@@ -234,8 +234,8 @@ __device__ __forceinline__ void mma_16816(float& d0, float& d1, float& d2, float
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c2), "f"(c3));
 }
 
-size_t gemv_mma_smem_bytes(int C) {
-  return (size_t)kGemvTok * (C + 8) * sizeof(uint16_t) + (size_t)kMmaRows * (C / 32);
+size_t gemv_mma_smem_bytes(int C, int warps) {
+  return (size_t)kGemvTok * (C + 8) * sizeof(uint16_t) + (size_t)16 * warps * (C / 32);
 }
 
 struct MmaGroup {
@@ -290,7 +290,9 @@ __device__ __forceinline__ void mma_compute(const MmaGroup& G, int b0, int KB, b
 // expert (rows past R idle). Shared memory holds the pass's tokens in f16
 // (8 x C, rows padded by 16 bytes) and the block's scale bytes.
 template <bool kGateUp>
-__global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(mma_warps(kGateUp) * 32) gemv_mma_kernel(GemvArgs a) {
+  constexpr int kMmaWarps = mma_warps(kGateUp);
+  constexpr int kMmaRows = 16 * kMmaWarps;
   pdl_wait_and_trigger();
   extern __shared__ __align__(16) uint8_t gsm[];
   const int slotj = blockIdx.y;
@@ -791,11 +793,12 @@ cudaError_t launch_gemv_v(const GemvArgs& a, int sm_count, cudaStream_t st) {
 
 cudaError_t configure_gemv(int Cmax) {
   const size_t smem = gemv_smem_bytes(Cmax);
-  const size_t smem_mma = gemv_mma_smem_bytes(Cmax);
+  const size_t smem_mma_gu = gemv_mma_smem_bytes(Cmax, kMmaWarpsGateUp);
+  const size_t smem_mma_dn = gemv_mma_smem_bytes(Cmax, kMmaWarpsDown);
   cudaError_t err = raise_smem_limit((const void*)gemv_kernel<true>, smem);
   if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_kernel<false>, smem);
-  if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<true>, smem_mma);
-  if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<false>, smem_mma);
+  if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<true>, smem_mma_gu);
+  if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_mma_kernel<false>, smem_mma_dn);
   const size_t smem_v = gemv_v_smem_bytes(Cmax);
   if (smem_v <= kSmemLimit) {  // larger rows fall back to variant 1
     if (err == cudaSuccess) err = raise_smem_limit((const void*)gemv_v_kernel<true>, smem_v);
@@ -807,10 +810,10 @@ cudaError_t configure_gemv(int Cmax) {
 cudaError_t launch_gemv_gateup(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st) {
   if (variant == 2 && gemv_v_smem_bytes(a.C) <= kSmemLimit) return launch_gemv_v<true>(a, sm_count, st);
   if (variant == 1) {
-    dim3 grid((a.R + kMmaRows - 1) / kMmaRows, max_touched);
+    dim3 grid((a.R + 16 * kMmaWarpsGateUp - 1) / (16 * kMmaWarpsGateUp), max_touched);
     {
-    const cudaError_t e_ =
-        launch_pdl(gemv_mma_kernel<true>, grid, dim3(kMmaWarps * 32), gemv_mma_smem_bytes(a.C), st, a);
+    const cudaError_t e_ = launch_pdl(gemv_mma_kernel<true>, grid, dim3(kMmaWarpsGateUp * 32),
+                                      gemv_mma_smem_bytes(a.C, kMmaWarpsGateUp), st, a);
     if (e_ != cudaSuccess) return e_;
   }
   } else {
@@ -826,10 +829,10 @@ cudaError_t launch_gemv_gateup(const GemvArgs& a, int max_touched, int variant, 
 cudaError_t launch_gemv_down(const GemvArgs& a, int max_touched, int variant, int sm_count, cudaStream_t st) {
   if (variant == 2 && gemv_v_smem_bytes(a.C) <= kSmemLimit) return launch_gemv_v<false>(a, sm_count, st);
   if (variant == 1) {
-    dim3 grid((a.R + kMmaRows - 1) / kMmaRows, max_touched);
+    dim3 grid((a.R + 16 * kMmaWarpsDown - 1) / (16 * kMmaWarpsDown), max_touched);
     {
-    const cudaError_t e_ =
-        launch_pdl(gemv_mma_kernel<false>, grid, dim3(kMmaWarps * 32), gemv_mma_smem_bytes(a.C), st, a);
+    const cudaError_t e_ = launch_pdl(gemv_mma_kernel<false>, grid, dim3(kMmaWarpsDown * 32),
+                                      gemv_mma_smem_bytes(a.C, kMmaWarpsDown), st, a);
     if (e_ != cudaSuccess) return e_;
   }
   } else {
