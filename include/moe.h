@@ -210,6 +210,18 @@ moe_status_t moe_debug_decode_codes(const uint8_t* bytes, int n, uint32_t* out_f
 moe_status_t moe_debug_route(moe_handle_t h, const void* x, const float* router_w, const float* router_b, int T,
                              int* idx, float* w, int* perm, int* offsets, void* stream);
 
+/*
+ * Test hook for the failure path of the bounded device-side waits (the pages
+ * have no counterpart): one thread of one block waits, with the same bounded
+ * wait the layer's kernels use, on a shared-memory barrier that nothing ever
+ * completes. After limit_us microseconds (1 <= limit_us <= 10000000) the wait
+ * gives up and raises the handle's status word, which the next
+ * moe_sync_status(h) reports as MOE_ERR_DEVICE_TIMEOUT (and clears). No copy or
+ * MMA is in flight, so the kernel returns normally and the context stays
+ * usable. Asynchronous on `stream`.
+ */
+moe_status_t moe_debug_wait_timeout(moe_handle_t h, long long limit_us, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

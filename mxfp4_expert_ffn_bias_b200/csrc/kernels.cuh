@@ -58,6 +58,7 @@ __global__ void combine_kernel(const float* __restrict__ slot, int T, int H, int
 __global__ void debug_dequant_kernel(const uint8_t* __restrict__ blocks, const uint8_t* __restrict__ scales,
                                      int rows, int cols, uint16_t* __restrict__ out);
 __global__ void debug_decode_codes_kernel(const uint8_t* __restrict__ bytes, int n, uint32_t* __restrict__ out);
+__global__ void debug_wait_timeout_kernel(unsigned* status, long long limit_us);
 
 // Decode path (routed-expert GEMVs on the CUDA cores).
 struct GemvArgs {

@@ -496,6 +496,14 @@ MOE_API moe_status_t moe_debug_decode_codes(const uint8_t* bytes, int n, uint32_
   return from_cuda(cudaGetLastError());
 }
 
+MOE_API moe_status_t moe_debug_wait_timeout(moe_handle_t h, long long limit_us, void* stream) {
+  if (!h || limit_us < 1 || limit_us > 10000000) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  h->last_stream = st;
+  debug_wait_timeout_kernel<<<1, 32, 0, st>>>(h->ws.status, limit_us);
+  return from_cuda(cudaGetLastError());
+}
+
 MOE_API moe_status_t moe_debug_route(moe_handle_t h, const void* x, const float* rw, const float* rb, int T,
                                      int* idx, float* w, int* perm, int* offsets, void* stream) {
   if (!h || !x || !rw || !rb || T < 1 || T > h->max_T) return MOE_ERR_INVALID_ARG;

@@ -1,6 +1,6 @@
 // Router (logits + top-k + softmax over k), the deterministic counting-sort
 // permutation of (token, slot) pairs by expert, the row gather for the grouped
-// GEMMs, the fixed-order slot combine, and two test-hook kernels.
+// GEMMs, the fixed-order slot combine, and three test-hook kernels.
 #include "common.cuh"
 #include "kernels.cuh"
 #include "mx_dequant.cuh"
@@ -964,6 +964,20 @@ __global__ void debug_dequant_kernel(const uint8_t* __restrict__ blocks, const u
     const uint32_t s = scales[(size_t)r * nb + b];
     *reinterpret_cast<uint4*>(out + (size_t)r * cols + cc * 8) = mx_dequant8_bf16(w, s);
   }
+}
+
+// One thread waits (bounded) on a barrier that is never completed: the wait gives up after limit_us and raises
+// the status word, exactly as a stalled wait inside the layer's kernels does. Nothing asynchronous is in flight.
+__global__ void debug_wait_timeout_kernel(unsigned* status, long long limit_us) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bar(&bar, 0, limit_us, &abort_flag, status);
 }
 
 __global__ void debug_decode_codes_kernel(const uint8_t* __restrict__ bytes, int n, uint32_t* __restrict__ out) {

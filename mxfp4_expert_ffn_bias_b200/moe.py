@@ -57,6 +57,7 @@ SIGNATURES = {
     "moe_debug_dequant": (_I, [_P, _P, _I, _I, _P, _P]),
     "moe_debug_decode_codes": (_I, [_P, _I, _P, _P]),
     "moe_debug_route": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
+    "moe_debug_wait_timeout": (_I, [_P, ctypes.c_longlong, _P]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _fn = getattr(_lib, _name)
@@ -160,6 +161,10 @@ def moe_debug_route(h, x, router_w, router_b, T: int, idx=None, w=None, perm=Non
                     stream=None) -> None:
     _check(_lib.moe_debug_route(h, _ptr(x), _ptr(router_w), _ptr(router_b), int(T), _ptr(idx), _ptr(w), _ptr(perm),
                                 _ptr(offsets), _stream(stream)), "moe_debug_route")
+
+
+def moe_debug_wait_timeout(h, limit_us: int, stream=None) -> None:
+    _check(_lib.moe_debug_wait_timeout(h, int(limit_us), _stream(stream)), "moe_debug_wait_timeout")
 
 
 class MoeLayer:

@@ -325,6 +325,30 @@ def test_invalid_token_counts_rejected(moe):
         moe.moe_destroy(h)
 
 
+def test_device_wait_timeout_reported_and_handle_recovers(moe):
+    # a bounded wait on a barrier that nothing completes gives up, the status word reports it once, and the
+    # same handle (same context) then runs the layer correctly
+    cfg = CONFIGS["tiny"]
+    inp = inputs_for("tiny")
+    dev = to_device(inp)
+    T = inp["x"].shape[0]
+    h = moe.moe_create(cfg.H, cfg.I, cfg.E, cfg.k, T)
+    try:
+        with pytest.raises(moe.MoeError) as ei:
+            moe.moe_debug_wait_timeout(h, 0)
+        assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+        moe.moe_debug_wait_timeout(h, 2000)
+        assert moe.moe_sync_status(h) == moe.MOE_ERR_DEVICE_TIMEOUT
+        assert moe.moe_sync_status(h) == moe.MOE_OK
+        out = run_forward(moe, h, dev, T, cfg.H)
+        torch.cuda.synchronize()
+        assert moe.moe_sync_status(h) == moe.MOE_OK
+    finally:
+        moe.moe_destroy(h)
+    ref, _, _ = oracle.moe_forward(inp, cfg.k, threads=NCPU)
+    assert_parity(bf16_dev_to_f64(out), ref, "tiny after a device wait timeout")
+
+
 def test_stage_times_reported(moe):
     cfg = CONFIGS["tiny"]
     dev = to_device(inputs_for("tiny"))
