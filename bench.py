@@ -110,9 +110,9 @@ _GEMV_TU = ["mxfp4_expert_ffn_bias_b200/csrc/gemv.cu", "mxfp4_expert_ffn_bias_b2
 _GEMM_TU = ["mxfp4_expert_ffn_bias_b200/csrc/gemm_sm100.cu"] + _GEMV_TU[1:]
 TRAFFIC = {
     # profiles/decode-kernels_gpt-oss-20b-decode.md: 194.24 MB read + 5.55 MB written
-    ("moe::gemv_mma_kernel<true>", "gpt-oss-20b-decode"): {"bytes": 199787520, "files": _GEMV_TU, "hash": "ba40c91127ef9c21"},
+    ("moe::gemv_mma_kernel<true>", "gpt-oss-20b-decode"): {"bytes": 199787520, "files": _GEMV_TU, "hash": "3c3db453abc33793"},
     # profiles/prefill-kernels_gpt-oss-20b-prefill.md: 376.81 MB read + 82.16 MB written
-    ("moe::grouped_mxfp4_gemm<true>", "gpt-oss-20b-prefill"): {"bytes": 458969088, "files": _GEMM_TU, "hash": "2d304a3f9878b4a8"},
+    ("moe::grouped_mxfp4_gemm<true>", "gpt-oss-20b-prefill"): {"bytes": 458969088, "files": _GEMM_TU, "hash": "0cd7e12f8fe98ac7"},
 }
 
 
