@@ -1,5 +1,6 @@
 """Host-side logic of bench.py that needs no GPU: the max-over-ranks reduction on two gloo ranks,
-the whole-job throughput, the algorithmic units, and the reference arm launched on two ranks."""
+the whole-job throughput, the algorithmic units, the reference arm launched on two ranks, and the rule
+that a stored DRAM traffic figure is reported only while its kernel sources are unchanged."""
 
 import json
 import os
@@ -72,3 +73,17 @@ def test_reference_arm_on_two_ranks_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_traffic_reported_only_while_sources_match(tmp_path, monkeypatch):
+    # a stored DRAM traffic figure belongs to the kernel sources it was captured from: it is reported while
+    # they hash the same and dropped (None) as soon as any of them changes
+    src = tmp_path / "k.cu"
+    src.write_text("kernel A\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    key = ("moe::k", "w")
+    monkeypatch.setitem(bench.TRAFFIC, key, {"bytes": 123, "files": ["k.cu"], "hash": bench._tu_hash(["k.cu"])})
+    assert bench.traffic_for(*key) == 123
+    src.write_text("kernel B\n")
+    assert bench.traffic_for(*key) is None
+    assert bench.traffic_for("moe::unknown", "w") is None
